@@ -1,0 +1,257 @@
+"""Plain fp64 CPU oracle for exact softmax attention and its analytic backward.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or link
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` use it. It shares no code with the CUDA library and imports
+nothing from the ``exact_io_aware_61_b200`` package.
+
+What it computes (and where the pages define it):
+
+* Scores ``S = Q K^T / sqrt(d)`` -- mentria.ai "Exact attention, sped up by
+  never writing the giant grid down", section "So don't load it all. Work one
+  block at a time." (block score equation). The scale is an explicit argument.
+* The optional mask, applied to the scores before the softmax --
+  fanfani.net "FlashAttention", section "The bottleneck was never the
+  arithmetic". The pages do not define the mask; the reading taken here is the
+  causal one: key ``j`` is visible to query ``i`` iff ``j <= i`` (square,
+  top-left aligned).
+* The max-subtracted softmax of each full score row -- mentria.ai, section
+  "But softmax needs the whole row at once." (safe-softmax equation).
+* ``O = P V`` and the per-row log-sum-exp ``LSE = m + ln(l)`` of the scaled
+  scores, the statistics the forward keeps for the backward -- fanfani.net,
+  section "The backward pass, and where the memory saving comes from";
+  synthetic.wiki "FlashAttention: attention's bottleneck is the wire, not the
+  maths", section "The backward pass buys memory with recompute".
+* The blockwise online-softmax pass (running max ``m``, running normaliser
+  ``l``, running output ``o``, each rescaled by ``exp(m_old - m_new)``) --
+  fanfani.net, section "A pinch of math: making the softmax work in pieces";
+  mentria.ai, section "The trick: keep a running max, and rebase as you go.".
+  It exists here only to pin the full-row oracle against the pages' claim that
+  the blockwise result is the same answer.
+* The backward pass. The pages only say that the score blocks are recomputed
+  from Q, K and the saved statistics; the gradient itself is the textbook
+  derivative of the softmax definition above:
+  ``dV = P^T dO``, ``dP = dO V^T``, ``D = rowsum(dO * O)``,
+  ``dS = P * (dP - D)``, ``dQ = scale dS K``, ``dK = scale dS^T Q``.
+
+Grouped-query attention (synthetic.wiki, section "Versions, and what the
+numbers say", names MQA/GQA without a head mapping): query head ``h`` reads
+KV head ``h // (Hq // Hkv)``; dK and dV sum over the query heads of a group.
+
+A row with no visible key (impossible for the square causal mask, kept for
+completeness) gets ``O = 0`` and ``LSE = -inf``.
+
+Layouts: Q, O, dO, dQ are ``[B, Hq, N, d]``; K, V, dK, dV are
+``[B, Hkv, N, d]``; LSE and D are ``[B, Hq, N]``. All arithmetic is float64.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "kv_head_of",
+    "masked_scores",
+    "softmax_rows",
+    "attention_probs",
+    "attention_forward",
+    "attention_forward_rows",
+    "online_softmax_forward",
+    "attention_backward",
+    "score_matrix_bytes",
+]
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def kv_head_of(hq: int, Hq: int, Hkv: int) -> int:
+    """KV head read by query head ``hq``: contiguous groups of ``Hq // Hkv``."""
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return hq // (Hq // Hkv)
+
+
+def masked_scores(q_bh, k_bh, scale: float, causal: bool, rows=None) -> np.ndarray:
+    """Scaled scores ``scale * Q K^T`` of one head, masked entries set to -inf.
+
+    ``q_bh`` is ``[N, d]`` (or ``[len(rows), d]`` when ``rows`` lists the query
+    positions it holds), ``k_bh`` is ``[N, d]``. Returns ``[n_rows, N]``.
+    """
+    q_bh = _f64(q_bh)
+    k_bh = _f64(k_bh)
+    n_keys = k_bh.shape[0]
+    s = scale * (q_bh @ k_bh.T)
+    if causal:
+        qpos = np.arange(q_bh.shape[0]) if rows is None else np.asarray(rows)
+        kpos = np.arange(n_keys)
+        s = np.where(kpos[None, :] <= qpos[:, None], s, -np.inf)
+    return s
+
+
+def softmax_rows(s: np.ndarray):
+    """Max-subtracted softmax of every row of ``s``.
+
+    Returns ``(P, m, l)`` with ``m`` the row maximum and ``l`` the sum of
+    ``exp(s - m)``, so that ``P = exp(s - m) / l``. Rows that are entirely
+    -inf give ``P = 0``, ``m = -inf``, ``l = 0``.
+    """
+    m = np.max(s, axis=-1)
+    finite = np.isfinite(m)
+    m_safe = np.where(finite, m, 0.0)
+    e = np.exp(s - m_safe[..., None])  # exp(-inf) = 0 for masked entries
+    l = np.sum(e, axis=-1)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        p = np.where(finite[..., None], e / np.where(finite, l, 1.0)[..., None], 0.0)
+    l = np.where(finite, l, 0.0)
+    return p, m, l
+
+
+def _lse(m, l):
+    with np.errstate(divide="ignore"):
+        return np.where(l > 0, m + np.log(np.where(l > 0, l, 1.0)), -np.inf)
+
+
+def attention_probs(q, k, scale: float, causal: bool) -> np.ndarray:
+    """Full attention-weight tensor ``P`` of shape ``[B, Hq, N, N]``."""
+    q = _f64(q)
+    k = _f64(k)
+    B, Hq, N, _ = q.shape
+    Hkv = k.shape[1]
+    p = np.empty((B, Hq, N, N))
+    for b in range(B):
+        for h in range(Hq):
+            s = masked_scores(q[b, h], k[b, kv_head_of(h, Hq, Hkv)], scale, causal)
+            p[b, h] = softmax_rows(s)[0]
+    return p
+
+
+def attention_forward(q, k, v, scale: float, causal: bool):
+    """Exact attention, materialising each head's N x N score matrix.
+
+    Returns ``(O [B,Hq,N,d], LSE [B,Hq,N])`` in float64.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    o = np.empty((B, Hq, N, v.shape[-1]))
+    lse = np.empty((B, Hq, N))
+    for b in range(B):
+        for h in range(Hq):
+            hk = kv_head_of(h, Hq, Hkv)
+            s = masked_scores(q[b, h], k[b, hk], scale, causal)
+            p, m, l = softmax_rows(s)
+            o[b, h] = p @ v[b, hk]
+            lse[b, h] = _lse(m, l)
+    return o, lse
+
+
+def attention_forward_rows(q, k, v, scale: float, causal: bool, b: int, h: int, rows):
+    """Exact attention for the listed query positions of one (batch, head).
+
+    Same definition as :func:`attention_forward`, restricted to the query
+    positions ``rows`` of batch ``b``, query head ``h``; used to check sampled
+    rows of workloads too large to materialise whole. Returns
+    ``(O_rows [len(rows), d], LSE_rows [len(rows)])``.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    Hq = np.shape(q)[1]
+    Hkv = np.shape(k)[1]
+    hk = kv_head_of(h, Hq, Hkv)
+    q_rows = _f64(np.asarray(q)[b, h][rows])
+    k_bh = _f64(np.asarray(k)[b, hk])
+    v_bh = _f64(np.asarray(v)[b, hk])
+    s = masked_scores(q_rows, k_bh, scale, causal, rows=rows)
+    p, m, l = softmax_rows(s)
+    return p @ v_bh, _lse(m, l)
+
+
+def online_softmax_forward(q, k, v, scale: float, causal: bool, block: int):
+    """Blockwise online-softmax attention in float64, keys taken ``block`` at a time.
+
+    Per query row it carries the running maximum ``m``, the running normaliser
+    ``l`` and the running weighted sum ``o``. For each key block with block
+    maximum ``m_blk``: ``m_new = max(m, m_blk)``, ``alpha = exp(m - m_new)``
+    (0 while ``m`` is still -inf), ``l = alpha l + sum exp(s - m_new)``,
+    ``o = alpha o + sum exp(s - m_new) v``. After the last block ``O = o / l``
+    once, and ``LSE = m + ln l``. The last block may be shorter than ``block``.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    dv = v.shape[-1]
+    o_out = np.empty((B, Hq, N, dv))
+    lse_out = np.empty((B, Hq, N))
+    for b in range(B):
+        for h in range(Hq):
+            hk = kv_head_of(h, Hq, Hkv)
+            m = np.full(N, -np.inf)
+            l = np.zeros(N)
+            o = np.zeros((N, dv))
+            for j0 in range(0, N, block):
+                j1 = min(j0 + block, N)
+                s = scale * (q[b, h] @ k[b, hk, j0:j1].T)
+                if causal:
+                    qpos = np.arange(N)[:, None]
+                    kpos = np.arange(j0, j1)[None, :]
+                    s = np.where(kpos <= qpos, s, -np.inf)
+                m_blk = np.max(s, axis=1)
+                m_new = np.maximum(m, m_blk)
+                seen = np.isfinite(m_new)
+                m_ref = np.where(seen, m_new, 0.0)
+                with np.errstate(invalid="ignore"):
+                    alpha = np.where(np.isfinite(m), np.exp(m - m_ref), 0.0)
+                e = np.exp(s - m_ref[:, None])
+                l = alpha * l + e.sum(axis=1)
+                o = alpha[:, None] * o + e @ v[b, hk, j0:j1]
+                m = m_new
+            with np.errstate(invalid="ignore", divide="ignore"):
+                o_out[b, h] = np.where(l[:, None] > 0, o / np.where(l > 0, l, 1.0)[:, None], 0.0)
+            lse_out[b, h] = _lse(m, l)
+    return o_out, lse_out
+
+
+def attention_backward(q, k, v, do, scale: float, causal: bool):
+    """Analytic gradients of ``O = softmax(scale Q K^T [+mask]) V``.
+
+    Given the upstream gradient ``dO`` returns ``(dQ, dK, dV, D)`` where
+    ``D = rowsum(dO * O)`` is the per-row term of the softmax Jacobian.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    do = _f64(do)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    D = np.empty((B, Hq, N))
+    for b in range(B):
+        for h in range(Hq):
+            hk = kv_head_of(h, Hq, Hkv)
+            s = masked_scores(q[b, h], k[b, hk], scale, causal)
+            p = softmax_rows(s)[0]
+            o = p @ v[b, hk]
+            dv[b, hk] += p.T @ do[b, h]
+            dp = do[b, h] @ v[b, hk].T
+            D[b, h] = np.sum(do[b, h] * o, axis=1)
+            ds = score_gradient(p, dp, D[b, h])
+            dq[b, h] = scale * (ds @ k[b, hk])
+            dk[b, hk] += scale * (ds.T @ q[b, h])
+    return dq, dk, dv, D
+
+
+def score_gradient(p, dp, D):
+    """Gradient with respect to the (pre-softmax) scores: ``P * (dP - D)``."""
+    return p * (dp - D[:, None])
+
+
+def score_matrix_bytes(N: int, heads: int, bytes_per_element: int) -> int:
+    """Bytes the unfused path would need to hold the N x N scores of ``heads`` heads."""
+    return N * N * heads * bytes_per_element
