@@ -1,0 +1,168 @@
+"""ctypes binding of ``libfa_b200.so`` (the C ABI in ``include/fa.h``).
+
+Argument marshalling only: every step of the attention computation runs in
+the CUDA kernels behind ``fa_fwd`` / ``fa_bwd``. PyTorch supplies device
+memory and the current stream. There is no CPU or library fallback: if the
+shared library is missing or cannot be loaded, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
+
+FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+FA_BF16, FA_F32 = 0, 1
+
+EXPORTED = (
+    "fa_fwd",
+    "fa_bwd",
+    "fa_bwd_workspace_size",
+    "fa_status_string",
+    "fa_last_device_status",
+    "fa_set_wait_timeout_ns",
+    "fa_selftest_wait_timeout",
+)
+
+_lock = threading.Lock()
+_handle = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library once and declare every exported signature."""
+    global _handle
+    with _lock:
+        if _handle is not None:
+            return _handle
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"CUDA library {path} is missing: build it with "
+                "`python -m exact_io_aware_61_b200.build` (no CPU fallback exists)")
+        lib = ctypes.CDLL(path)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+        lib.fa_fwd.restype = i
+        lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp]
+        lib.fa_bwd.restype = i
+        lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i]
+        lib.fa_bwd_workspace_size.restype = sz
+        lib.fa_status_string.argtypes = [i]
+        lib.fa_status_string.restype = ctypes.c_char_p
+        lib.fa_last_device_status.argtypes = [vp]
+        lib.fa_last_device_status.restype = i
+        lib.fa_set_wait_timeout_ns.argtypes = [ctypes.c_longlong]
+        lib.fa_set_wait_timeout_ns.restype = None
+        lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
+        lib.fa_selftest_wait_timeout.restype = i
+        _handle = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float32:
+        return FA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: bf16 or float32 tensors expected")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_tensor(name, t, device):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (dense BHND layout)")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """Call ``fa_fwd`` on existing tensors: q [B,Hq,N,d], k/v [B,Hkv,N,d], o like q, lse [B,Hq,N] f32."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse)):
+        _check_tensor(name, t, q.device)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    rc = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, float(scale),
+                       int(bool(causal)), _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd")
+
+
+def fa_bwd_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
+    return int(load().fa_bwd_workspace_size(B, Hq, Hkv, N, d))
+
+
+def fa_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool, scale: float, stream=None) -> None:
+    """Call ``fa_bwd`` on existing tensors; ``workspace`` is a uint8 CUDA tensor."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse), ("do", do), ("dq", dq),
+                    ("dk", dk), ("dv", dv)):
+        _check_tensor(name, t, q.device)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    ws_ptr = None if workspace is None else ctypes.c_void_p(workspace.data_ptr())
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                       ws_ptr, ws_bytes, B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _dtype_code(q),
+                       ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd")
+
+
+def forward(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """Allocate O and LSE with torch and run ``fa_fwd``. Returns ``(o, lse)``."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, stream=None):
+    """Allocate dQ, dK, dV and the workspace with torch and run ``fa_bwd``."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    B, Hq, N, d = q.shape
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    ws = torch.empty(max(fa_bwd_workspace_size(B, Hq, k.shape[1], N, d), 16), dtype=torch.uint8, device=q.device)
+    fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal, scale, stream)
+    return dq, dk, dv
+
+
+def fa_last_device_status(stream=None) -> int:
+    return int(load().fa_last_device_status(ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def fa_set_wait_timeout_ns(ns: int) -> None:
+    load().fa_set_wait_timeout_ns(int(ns))
+
+
+def fa_selftest_wait_timeout(ns: int, stream=None) -> int:
+    return int(load().fa_selftest_wait_timeout(int(ns), ctypes.c_void_p(_stream_ptr(stream))))

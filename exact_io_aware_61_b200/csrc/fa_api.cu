@@ -1,0 +1,329 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument checks, TMA
+// tensor maps, kernel selection and launches. One translation unit holds
+// every kernel so that they share the device status word.
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "sm100_ptx.cuh"
+#include "fwd_sm100.cuh"
+#include "fwd_f32.cuh"
+#include "bwd_sm100.cuh"
+
+namespace {
+
+constexpr long long kDefaultTimeoutNs = 2000000000LL;
+std::atomic<long long> g_timeout_ns{kDefaultTimeoutNs};
+
+// Waits only on a barrier nothing arrives at: the bounded wait must run out.
+__global__ void fa_selftest_wait_kernel(unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    fa::mbar_init(fa::smem_u32(&bar), 1);
+    fa::fence_mbar_init();
+  }
+  __syncthreads();
+  fa::WaitCtl wc{&abort_flag, timeout_ns};
+  if (threadIdx.x == 0) (void)fa::mbar_wait(fa::smem_u32(&bar), 0, wc);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// The kernels are built for sm_100a only: CC 10.0.
+int check_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  return FA_OK;
+}
+
+// Opt every kernel into its dynamic shared memory, once per device.
+int prepare_kernels(int dev) {
+  static std::mutex mu;
+  static bool done[128] = {};
+  if (dev < 0 || dev >= 128) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev]) return FA_OK;
+  cudaError_t e = cudaSuccess;
+  auto set = [&](const void* fn, int bytes) {
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  };
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<64>), fa::FwdCfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<128>), fa::FwdCfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<256>), fa::FwdCfg<256>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<64>), fa::fwd_f32_smem_bytes<64>());
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<128>), fa::fwd_f32_smem_bytes<128>());
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<256>), fa::fwd_f32_smem_bytes<256>());
+  set(reinterpret_cast<const void*>(&fa::fa_bwd_main_kernel<64>), fa::BwdCfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd_main_kernel<128>), fa::BwdCfg<128>::SMEM_BYTES);
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  done[dev] = true;
+  return FA_OK;
+}
+
+// Rank-3 tiled map over a dense [outer][rows][inner] tensor with a
+// (box_inner x box_rows x 1) box and 128-byte swizzle; out-of-bounds reads
+// fill zeros, out-of-bounds writes are dropped.
+int make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType type, uint64_t elem_bytes, uint64_t inner,
+             uint64_t rows, uint64_t outer, uint32_t box_inner, uint32_t box_rows) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return FA_ERR_CUDA;
+  const cuuint64_t dims[3] = {inner, rows, outer};
+  const cuuint64_t strides[2] = {inner * elem_bytes, inner * rows * elem_bytes};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = encode(map, type, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared shape checks. Returns FA_OK, or the error to report.
+int check_shape(int B, int Hq, int Hkv, int N, int d, float scale, int causal, int dtype) {
+  if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || d < 1) return FA_ERR_INVALID;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_INVALID;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  // TMA coordinates and tile indices are 32-bit.
+  if (static_cast<long long>(B) * Hq > INT32_MAX / 2 || N > INT32_MAX - 256) return FA_ERR_INVALID;
+  return FA_OK;
+}
+
+unsigned long long timeout_now() { return static_cast<unsigned long long>(g_timeout_ns.load()); }
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+template <int HD>
+int launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                    int N, float scale, int causal, cudaStream_t stream) {
+  using C = fa::FwdCfg<HD>;
+  CUtensorMap mq, mk, mv;
+  int rc = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hq, 64, 128);
+  if (rc == FA_OK)
+    rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  if (rc == FA_OK)
+    rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  if (rc != FA_OK) return rc;
+  fa::FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.num_q_tiles = (N + C::BM - 1) / C::BM;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.timeout_ns = timeout_now();
+  const long long blocks = static_cast<long long>(p.num_q_tiles) * B * Hq;
+  if (blocks > INT32_MAX) return FA_ERR_INVALID;
+  fa::fa_fwd_bf16_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+template <int HD>
+int launch_fwd_f32(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                   float scale, int causal, cudaStream_t stream) {
+  fa::FwdF32Params p;
+  p.q = static_cast<const float*>(q);
+  p.k = static_cast<const float*>(k);
+  p.v = static_cast<const float*>(v);
+  p.o = static_cast<float*>(o);
+  p.lse = lse;
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.scale = scale;
+  p.causal = causal;
+  const long long blocks = static_cast<long long>((N + 15) / 16) * B * Hq;
+  if (blocks > INT32_MAX) return FA_ERR_INVALID;
+  fa::fa_fwd_f32_kernel<HD><<<static_cast<unsigned>(blocks), 128, fa::fwd_f32_smem_bytes<HD>(), stream>>>(p);
+  return launch_status();
+}
+
+size_t padded_rows(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
+
+template <int HD>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+               void* dq, void* dk, void* dv, void* ws, int B, int Hq, int Hkv, int N, float scale, int causal,
+               cudaStream_t stream) {
+  using C = fa::BwdCfg<HD>;
+  const size_t npad = padded_rows(N);
+  const size_t rows_q = static_cast<size_t>(B) * Hq;
+  float* ws_delta = static_cast<float*>(ws);
+  float* ws_lse2 = ws_delta + rows_q * npad;
+  float* dq_acc = ws_lse2 + rows_q * npad;
+
+  fa::BwdPrepParams pp;
+  pp.o = static_cast<const __nv_bfloat16*>(o);
+  pp.dO = static_cast<const __nv_bfloat16*>(dO);
+  pp.lse = lse;
+  pp.ws_delta = ws_delta;
+  pp.ws_lse2 = ws_lse2;
+  pp.dq_acc = dq_acc;
+  pp.N = N;
+  pp.Npad = static_cast<int>(npad);
+  const long long prep_blocks = static_cast<long long>(npad / 32) * static_cast<long long>(rows_q);
+  if (prep_blocks > INT32_MAX) return FA_ERR_INVALID;
+  fa::fa_bwd_prep_kernel<HD><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(pp);
+  int rc = launch_status();
+  if (rc != FA_OK) return rc;
+
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  rc = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
+  if (rc == FA_OK)
+    rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  if (rc == FA_OK)
+    rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  if (rc == FA_OK) rc = make_map(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
+  if (rc == FA_OK) rc = make_map(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, N, rows_q, 32, 128);
+  if (rc != FA_OK) return rc;
+
+  fa::BwdParams p;
+  p.ws_delta = ws_delta;
+  p.ws_lse2 = ws_lse2;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.N = N;
+  p.Npad = static_cast<int>(npad);
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.num_tiles = static_cast<int>(npad / 128);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.causal = causal;
+  p.timeout_ns = timeout_now();
+  const long long blocks = static_cast<long long>(p.num_tiles) * B * Hkv;
+  if (blocks > INT32_MAX) return FA_ERR_INVALID;
+  fa::fa_bwd_main_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
+                                                                                                    mdq, p);
+  rc = launch_status();
+  if (rc != FA_OK) return rc;
+
+  const size_t n4 = rows_q * static_cast<size_t>(N) * HD / 4;
+  const size_t want = (n4 + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
+  fa::fa_bwd_dq_kernel<<<grid, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n4);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID: return "FA_ERR_INVALID: invalid argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: not implemented for these arguments or this device";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a device-side bounded wait ran out";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
+    default: return "unknown fa_status";
+  }
+}
+
+void fa_set_wait_timeout_ns(long long timeout_ns) {
+  g_timeout_ns.store(timeout_ns > 0 ? timeout_ns : kDefaultTimeoutNs);
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
+           float scale, int causal, int dtype, fa_stream_t stream) {
+  int rc = check_shape(B, Hq, Hkv, N, d, scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (B == 0 || N == 0) return FA_OK;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID;
+  int dev = 0;
+  if ((rc = check_device(&dev)) != FA_OK) return rc;
+  if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == FA_BF16) {
+    switch (d) {
+      case 64: return launch_fwd_bf16<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
+      case 128: return launch_fwd_bf16<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
+      default: return launch_fwd_bf16<256>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
+    }
+  }
+  switch (d) {
+    case 64: return launch_fwd_f32<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
+    case 128: return launch_fwd_f32<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
+    default: return launch_fwd_f32<256>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
+  }
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || d < 1 || Hq % Hkv != 0) return 0;
+  const size_t rows_q = static_cast<size_t>(B) * Hq;
+  return sizeof(float) * (2 * rows_q * padded_rows(N) + rows_q * static_cast<size_t>(N) * d);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+           void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
+           float scale, int causal, int dtype, fa_stream_t stream) {
+  int rc = check_shape(B, Hq, Hkv, N, d, scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return FA_OK;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID;
+  if (workspace == nullptr || workspace_bytes < fa_bwd_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_INVALID;
+  int dev = 0;
+  if ((rc = check_device(&dev)) != FA_OK) return rc;
+  if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s);
+  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s);
+}
+
+int fa_last_device_status(fa_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  return v;
+}
+
+int fa_selftest_wait_timeout(long long timeout_ns, fa_stream_t stream) {
+  if (timeout_ns <= 0 || timeout_ns > 10000000000LL) return FA_ERR_INVALID;
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != FA_OK) return rc;
+  fa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(timeout_ns));
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,164 @@
+/*
+ * fa.h -- C ABI of the exact tiled-attention library for NVIDIA B200 (sm_100a).
+ *
+ * The library computes exact softmax attention
+ *     O = softmax(scale * Q K^T  [+ causal mask]) V
+ * tile by tile with the online-softmax recurrence (running maximum m, running
+ * normaliser l, running output rescaled by exp(m_old - m_new)), so the N x N
+ * score matrix never reaches device memory, and the training backward that
+ * keeps only O and the per-row log-sum-exp and recomputes the score tiles.
+ * Sources for the method:
+ *   - fanfani.net "FlashAttention": "Do not materialize the matrix" (tiling),
+ *     "A pinch of math: making the softmax work in pieces" (the recurrence and
+ *     the single division by l at the end), "The backward pass, and where the
+ *     memory saving comes from" (keep per-row statistics, recompute blocks);
+ *   - mentria.ai "Exact attention, sped up by never writing the giant grid
+ *     down": block score equation (S_ij = Q_i K_j^T / sqrt(d)), safe-softmax
+ *     equation, running-max recurrence;
+ *   - synthetic.wiki "FlashAttention: attention's bottleneck is the wire, not
+ *     the maths": "The backward pass buys memory with recompute"; "Versions,
+ *     and what the numbers say" (head dimensions up to 256, MQA/GQA).
+ *
+ * Conventions shared by every entry point
+ *   Layout   dense row-major "BHND": Q, O, dO, dQ are [B][Hq][N][d];
+ *            K, V, dK, dV are [B][Hkv][N][d]; LSE is float [B][Hq][N].
+ *   Heads    grouped-query attention: query head h reads KV head
+ *            h / (Hq / Hkv) (contiguous groups); Hkv == Hq is plain multi-head,
+ *            Hkv == 1 is multi-query.
+ *   Mask     causal != 0 hides key j from query i when j > i (square,
+ *            top-left aligned). The pages name "the mask" without defining
+ *            it; this is the reading the library implements.
+ *   LSE      natural-log log-sum-exp of the scaled scores of each row:
+ *            LSE_i = m_i + ln(l_i). It stands in for the two numbers per query
+ *            (m, l) that the pages keep: P = exp(scale*S - LSE) rebuilds the
+ *            weights without a second pass.
+ *   Pointers device pointers (cudaMalloc / torch CUDA tensors), each 16-byte
+ *            aligned. The caller owns every buffer; the library allocates no
+ *            device memory and keeps no per-call state.
+ *   Streams  every call enqueues its kernels on `stream` (0 = legacy default
+ *            stream) and returns without synchronising.
+ *   Errors   arguments are checked before anything is launched; on a
+ *            non-zero return nothing was launched and no output was written.
+ *            Kernels that hit a bounded wait limit record FA_ERR_TIMEOUT in a
+ *            per-device status word, read (and cleared) by
+ *            fa_last_device_status().
+ *   Empty    B == 0 or N == 0 is a valid empty problem: FA_OK, no launch.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; declared here so that the header
+ * does not need the CUDA headers. */
+typedef struct CUstream_st* fa_stream_t;
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID = 1,      /* bad argument: null/misaligned pointer, bad size */
+    FA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+    FA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out */
+    FA_ERR_WORKSPACE = 5     /* workspace missing or smaller than required */
+} fa_status;
+
+typedef enum {
+    FA_BF16 = 0,  /* bfloat16 tensors, float32 accumulation (tensor cores) */
+    FA_F32 = 1    /* float32 tensors, float32 arithmetic (CUDA cores) */
+} fa_dtype;
+
+/*
+ * fa_fwd -- forward pass: O and LSE.
+ *
+ *   q [B][Hq][N][d], k/v [B][Hkv][N][d]   inputs, element type `dtype`
+ *   o [B][Hq][N][d]                        output, element type `dtype`
+ *   lse [B][Hq][N]                         output, float32, natural log
+ *   d in {64, 128, 256}; Hq % Hkv == 0; B, N >= 0; Hq, Hkv >= 1
+ *   scale: the factor applied to Q K^T (1/sqrt(d) gives the pages' scores)
+ *   causal: 0 or 1
+ *   dtype: FA_BF16 (all d) or FA_F32 (all d)
+ * Computes, per (batch, query head), the fused tiled pass of "Do not
+ * materialize the matrix" with the recurrence of "A pinch of math", dividing
+ * by l once at the end. Returns fa_status.
+ */
+FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+           int dtype, fa_stream_t stream);
+
+/*
+ * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs: the
+ * per-row term D = rowsum(dO * O) and the log2-scaled LSE, both float32 and
+ * padded to a multiple of 128 rows per head, plus a float32 dQ accumulator
+ * [B][Hq][N][d]. Linear in N: nothing N x N is ever allocated. Returns 0 for
+ * invalid sizes.
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * fa_bwd -- backward pass: dQ, dK, dV from Q, K, V, O, LSE and dO.
+ *
+ *   q, o, dO [B][Hq][N][d], k, v [B][Hkv][N][d]   inputs (bf16)
+ *   lse [B][Hq][N] float32                          input, as written by fa_fwd
+ *   dq [B][Hq][N][d], dk, dv [B][Hkv][N][d]         outputs (bf16); dk and dv
+ *                                                   sum over each KV head's
+ *                                                   group of query heads
+ *   workspace, workspace_bytes                      scratch owned by the caller,
+ *                                                   >= fa_bwd_workspace_size()
+ *                                                   bytes, 16-byte aligned;
+ *                                                   contents on entry ignored
+ * Recomputes every score tile from Q and K and the stored LSE ("The backward
+ * pass, and where the memory saving comes from"): P = exp(scale*S - LSE),
+ * dV = P^T dO, dP = dO V^T, dS = P * (dP - D), dQ = scale dS K,
+ * dK = scale dS^T Q. Supports dtype FA_BF16 with d in {64, 128}; other
+ * combinations return FA_ERR_UNSUPPORTED. Three kernels run in stream order:
+ * D and LSE preparation (and zeroing of the dQ accumulator), the main
+ * recompute kernel, and the dQ conversion.
+ */
+FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o,
+           const float* lse, const void* dO, void* dq, void* dk, void* dv,
+           void* workspace, size_t workspace_bytes,
+           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+           int dtype, fa_stream_t stream);
+
+/* Human-readable name of a fa_status value (static string, never NULL). */
+FA_API const char* fa_status_string(int status);
+
+/*
+ * fa_last_device_status -- synchronises `stream`, returns the current
+ * device's status word (FA_OK, or FA_ERR_TIMEOUT when some kernel gave up on
+ * a bounded wait since the last call) and clears it. FA_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+FA_API int fa_last_device_status(fa_stream_t stream);
+
+/*
+ * fa_set_wait_timeout_ns -- limit, in nanoseconds, on every spin-wait inside
+ * the kernels launched after this call (default 2e9 = 2 s). Values <= 0
+ * restore the default. Process-wide.
+ */
+FA_API void fa_set_wait_timeout_ns(long long timeout_ns);
+
+/*
+ * fa_selftest_wait_timeout -- launches one block that waits on a barrier
+ * nothing ever arrives at, with a limit of `timeout_ns`, so that the bounded
+ * wait runs out and records FA_ERR_TIMEOUT in the status word (read it with
+ * fa_last_device_status). Exercises the failure path without faulting or
+ * hanging the GPU. Returns FA_ERR_INVALID for timeout_ns outside (0, 1e10].
+ */
+FA_API int fa_selftest_wait_timeout(long long timeout_ns, fa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,104 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports
+every function ``include/fa.h`` declares, and rejects bad arguments before it
+touches the device. No kernel is launched here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_io_aware_61_b200 as fa
+from exact_io_aware_61_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return fa.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    return sorted(set(re.findall(r"FA_API\s+[\w\s\*]*?\b(fa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_status_string", "fa_last_device_status"):
+        assert must in names
+    assert sorted(fa.EXPORTED) == names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {fa.LIB_PATH}").read()
+    exported = set(re.findall(r" T (fa_\w+)", out))
+    assert set(_declared()) <= exported
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        s = fa.status_string(code)
+        assert s.startswith("FA_")
+    assert "unknown" in fa.status_string(99)
+
+
+def test_workspace_formula(lib):
+    # D and log2-scaled LSE padded to 128 rows per head, plus an f32 dQ accumulator
+    B, Hq, Hkv, N, d = 2, 16, 16, 4096, 128
+    assert fa.fa_bwd_workspace_size(B, Hq, Hkv, N, d) == 4 * (2 * B * Hq * 4096 + B * Hq * N * d)
+    assert fa.fa_bwd_workspace_size(1, 4, 2, 129, 64) == 4 * (2 * 4 * 256 + 4 * 129 * 64)
+    assert fa.fa_bwd_workspace_size(1, 3, 2, 64, 64) == 0  # Hq not a multiple of Hkv
+    # linear in N: nothing N x N
+    a = fa.fa_bwd_workspace_size(1, 1, 1, 8192, 128)
+    b = fa.fa_bwd_workspace_size(1, 1, 1, 16384, 128)
+    assert b == 2 * a
+
+
+def _fwd(lib, **kw):
+    args = dict(B=1, Hq=2, Hkv=2, N=64, d=64, scale=0.125, causal=0, dtype=0)
+    args.update(kw)
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    return lib.fa_fwd(p, p, p, p, p, args["B"], args["Hq"], args["Hkv"], args["N"], args["d"],
+                      args["scale"], args["causal"], args["dtype"], None)
+
+
+def test_validation_before_any_device_work(lib):
+    assert _fwd(lib, N=-1) == fa.FA_ERR_INVALID
+    assert _fwd(lib, B=-2) == fa.FA_ERR_INVALID
+    assert _fwd(lib, Hq=0) == fa.FA_ERR_INVALID
+    assert _fwd(lib, Hq=3, Hkv=2) == fa.FA_ERR_INVALID
+    assert _fwd(lib, d=96) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, causal=3) == fa.FA_ERR_INVALID
+    assert _fwd(lib, dtype=5) == fa.FA_ERR_INVALID
+    assert _fwd(lib, scale=float("inf")) == fa.FA_ERR_INVALID
+    assert _fwd(lib, B=0) == fa.FA_OK  # empty problem
+    assert _fwd(lib, N=0) == fa.FA_OK
+    # null pointers
+    assert lib.fa_fwd(None, None, None, None, None, 1, 1, 1, 8, 64, 0.1, 0, 0, None) == fa.FA_ERR_INVALID
+    # misaligned pointer
+    p, m = ctypes.c_void_p(64), ctypes.c_void_p(66)
+    assert lib.fa_fwd(p, p, m, p, p, 1, 1, 1, 8, 64, 0.1, 0, 0, None) == fa.FA_ERR_INVALID
+    # backward: f32 and d=256 are not implemented; short workspace
+    p = ctypes.c_void_p(64)
+    args = [p] * 9
+    assert lib.fa_bwd(*args, p, 1 << 30, 1, 1, 1, 8, 64, 0.1, 0, 1, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_bwd(*args, p, 1 << 30, 1, 1, 1, 8, 256, 0.1, 0, 0, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_bwd(*args, p, 16, 1, 1, 1, 8, 64, 0.1, 0, 0, None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_bwd(*args, None, 1 << 30, 1, 1, 1, 8, 64, 0.1, 0, 0, None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_selftest_wait_timeout(0, None) == fa.FA_ERR_INVALID
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from exact_io_aware_61_b200 import _lib
+    saved = _lib._handle
+    _lib._handle = None
+    try:
+        with pytest.raises(RuntimeError, match="missing"):
+            _lib.load(str(tmp_path / "nope.so"))
+    finally:
+        _lib._handle = saved

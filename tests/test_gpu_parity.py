@@ -1,0 +1,250 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Tolerances: float32 inputs, O and LSE max-abs <= 1e-5; bf16 inputs with fp32
+accumulation, O max-abs <= 2e-2 and LSE max-abs <= 1e-3; gradients dQ, dK, dV
+relative Frobenius error <= 2e-2. Inputs are the seeded synthetic tensors of
+``exact_io_aware_61_b200.inputs``; the oracle gets the same values in fp64.
+Full-size workloads are checked on sampled rows (forward) or sampled heads
+(backward) that the oracle computes one by one, plus properties that hold at
+any size.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.attention as ORACLE
+from exact_io_aware_61_b200 import inputs as INP
+
+pytestmark = pytest.mark.gpu
+
+O_TOL_F32, LSE_TOL_F32 = 1e-5, 1e-5
+O_TOL_BF16, LSE_TOL_BF16 = 2e-2, 1e-3
+GRAD_TOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def fa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    import exact_io_aware_61_b200 as fa_mod
+    fa_mod.load()  # raises if the library is missing: no fallback
+    return fa_mod
+
+
+def _to_dev(t):
+    return t.to("cuda").contiguous()
+
+
+def _run_fwd(fa, inp, causal, scale):
+    q, k, v = (_to_dev(inp[n]) for n in ("q", "k", "v"))
+    o, lse = fa.forward(q, k, v, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.FA_OK
+    return o, lse
+
+
+def _rel_fro(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+# ------------------------------------------------------------------ forward
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_f32_b1_h2_n256_d64(fa, seed, causal):
+    inp = INP.make_inputs(1, 2, 2, 256, 64, "f32", seed=seed)
+    o, lse = _run_fwd(fa, inp, causal, 1 / 8)
+    ro, rl = ORACLE.attention_forward(*(INP.as_f64(inp[n]) for n in "qkv"), 1 / 8, causal)
+    assert np.max(np.abs(INP.as_f64(o) - ro)) <= O_TOL_F32
+    assert np.max(np.abs(INP.as_f64(lse) - rl)) <= LSE_TOL_F32
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 2, 2, 1, 64), (1, 1, 1, 5, 128), (2, 3, 3, 127, 64), (1, 2, 1, 129, 128),
+    (1, 4, 2, 300, 64), (1, 2, 2, 300, 256), (2, 4, 1, 200, 128), (1, 1, 1, 1, 256),
+])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_f32_edge_shapes(fa, shape, causal):
+    B, Hq, Hkv, N, d = shape
+    inp = INP.make_inputs(B, Hq, Hkv, N, d, "f32", seed=11)
+    o, lse = _run_fwd(fa, inp, causal, d ** -0.5)
+    ro, rl = ORACLE.attention_forward(*(INP.as_f64(inp[n]) for n in "qkv"), d ** -0.5, causal)
+    assert np.max(np.abs(INP.as_f64(o) - ro)) <= O_TOL_F32
+    assert np.max(np.abs(INP.as_f64(lse) - rl)) <= LSE_TOL_F32
+
+
+BF16_EDGE = [
+    (1, 1, 1, 1, 64), (1, 2, 2, 1, 128), (1, 1, 1, 1, 256),
+    (1, 2, 2, 127, 64), (1, 2, 2, 128, 128), (1, 2, 2, 129, 128), (2, 3, 3, 300, 64),
+    (1, 4, 1, 257, 128), (1, 4, 2, 384, 256), (1, 2, 2, 640, 128), (1, 8, 2, 1000, 64),
+    (3, 2, 1, 513, 256),
+]
+
+
+@pytest.mark.parametrize("shape", BF16_EDGE, ids=lambda s: "b%d_h%d_kv%d_n%d_d%d" % s)
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_bf16_edge_shapes(fa, shape, causal):
+    B, Hq, Hkv, N, d = shape
+    inp = INP.make_inputs(B, Hq, Hkv, N, d, "bf16", seed=N + d)
+    o, lse = _run_fwd(fa, inp, causal, d ** -0.5)
+    ro, rl = ORACLE.attention_forward(*(INP.as_f64(inp[n]) for n in "qkv"), d ** -0.5, causal)
+    assert np.max(np.abs(INP.as_f64(o) - ro)) <= O_TOL_BF16
+    assert np.max(np.abs(INP.as_f64(lse) - rl)) <= LSE_TOL_BF16
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_bf16_b4_h16_n2048_d64(fa, causal):
+    w = INP.WORKLOADS["fwd_bf16_b4_h16_n2048_d64"]
+    inp = INP.workload_inputs(w, seed=1001)
+    o, lse = _run_fwd(fa, inp, causal, w.scale)
+    ro, rl = ORACLE.attention_forward(*(INP.as_f64(inp[n]) for n in "qkv"), w.scale, causal)
+    assert np.max(np.abs(INP.as_f64(o) - ro)) <= O_TOL_BF16
+    assert np.max(np.abs(INP.as_f64(lse) - rl)) <= LSE_TOL_BF16
+
+
+def _sample_rows(N, rng, n_random=24):
+    fixed = [0, 1, 2, 127, 128, 129, N // 2, N - 129, N - 128, N - 2, N - 1]
+    rows = set(r for r in fixed if 0 <= r < N)
+    rows.update(int(x) for x in rng.integers(0, N, n_random))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name", [
+    "fwd_causal_bf16_b2_h32_n8192_d128",
+    "gqa_causal_bf16_b1_h32_kv8_n16384_d128",
+    "gqa_causal_bf16_b1_h16_kv4_n8192_d256",
+])
+def test_fwd_bf16_full_size_sampled_rows(fa, name):
+    w = INP.WORKLOADS[name]
+    inp = INP.workload_inputs(w, seed=1000 + len(name))
+    o, lse = _run_fwd(fa, inp, True, w.scale)
+    o_h, lse_h = o.float().cpu().numpy(), lse.cpu().numpy()
+    q, k, v = (inp[n].float().numpy() for n in "qkv")
+    rng = np.random.default_rng(7)
+    worst_o = worst_l = 0.0
+    for b in range(w.B):
+        for h in range(w.Hq):
+            rows = _sample_rows(w.N, rng)
+            ro, rl = ORACLE.attention_forward_rows(q, k, v, w.scale, True, b, h, rows)
+            worst_o = max(worst_o, float(np.max(np.abs(o_h[b, h, rows] - ro))))
+            worst_l = max(worst_l, float(np.max(np.abs(lse_h[b, h, rows] - rl))))
+    assert worst_o <= O_TOL_BF16, worst_o
+    assert worst_l <= LSE_TOL_BF16, worst_l
+    assert np.all(np.isfinite(o_h)) and np.all(np.isfinite(lse_h))
+
+
+def test_fwd_bf16_deterministic(fa):
+    inp = INP.make_inputs(2, 4, 2, 1000, 128, "bf16", seed=5)
+    o1, l1 = _run_fwd(fa, inp, True, 0.09)
+    o2, l2 = _run_fwd(fa, inp, True, 0.09)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ----------------------------------------------------------------- backward
+
+def _run_bwd(fa, inp, causal, scale):
+    q, k, v, do = (_to_dev(inp[n]) for n in ("q", "k", "v", "do"))
+    o, lse = fa.forward(q, k, v, causal=causal, scale=scale)
+    dq, dk, dv = fa.backward(q, k, v, o, lse, do, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.FA_OK
+    return dq, dk, dv
+
+
+BWD_SHAPES = [
+    (1, 1, 1, 1, 64), (1, 2, 2, 100, 64), (1, 2, 2, 128, 128), (2, 2, 2, 257, 128),
+    (1, 4, 2, 300, 64), (1, 4, 1, 384, 128), (1, 2, 2, 1000, 128), (2, 6, 3, 513, 64),
+]
+
+
+@pytest.mark.parametrize("shape", BWD_SHAPES, ids=lambda s: "b%d_h%d_kv%d_n%d_d%d" % s)
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_bf16_shapes(fa, shape, causal):
+    B, Hq, Hkv, N, d = shape
+    inp = INP.make_inputs(B, Hq, Hkv, N, d, "bf16", seed=3 * N + d, grad=True)
+    dq, dk, dv = _run_bwd(fa, inp, causal, d ** -0.5)
+    rq, rk, rv, _ = ORACLE.attention_backward(*(INP.as_f64(inp[n]) for n in ("q", "k", "v", "do")),
+                                             d ** -0.5, causal)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        err = _rel_fro(INP.as_f64(got), ref)
+        assert err <= GRAD_TOL, (name, err)
+
+
+def test_bwd_train_causal_b2_h16_n4096_d128(fa):
+    w = INP.WORKLOADS["train_causal_bf16_b2_h16_n4096_d128"]
+    inp = INP.workload_inputs(w, seed=1005)
+    dq, dk, dv = _run_bwd(fa, inp, True, w.scale)
+    dq_h, dk_h, dv_h = (INP.as_f64(t) for t in (dq, dk, dv))
+    # property at full size: every row of P sums to one, so sum_j dV_j = sum_i dO_i
+    do = INP.as_f64(inp["do"])
+    lhs, rhs = dv_h.sum(axis=2), do.sum(axis=2)
+    assert _rel_fro(lhs, rhs) <= GRAD_TOL
+    # full oracle on sampled heads
+    q, k, v = (INP.as_f64(inp[n]) for n in "qkv")
+    for b, h in ((0, 0), (0, 7), (1, 3), (1, 15)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        rq, rk, rv, _ = ORACLE.attention_backward(q[sl], k[sl], v[sl], do[sl], w.scale, True)
+        for name, got, ref in (("dq", dq_h[sl], rq), ("dk", dk_h[sl], rk), ("dv", dv_h[sl], rv)):
+            err = _rel_fro(got, ref)
+            assert err <= GRAD_TOL, (name, b, h, err)
+
+
+# ---------------------------------------------------------- ABI behaviour
+
+def test_abi_rejects_bad_arguments_without_writing(fa):
+    q = torch.randn(1, 2, 64, 64, device="cuda").to(torch.bfloat16)
+    k, v = q.clone(), q.clone()
+    o = torch.full_like(q, 7.0)
+    lse = torch.full((1, 2, 64), 7.0, device="cuda")
+
+    import ctypes
+
+    def ptr(t):
+        return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+    def call(**kw):
+        args = dict(q=q, k=k, v=v, o=o, lse=lse, B=1, Hq=2, Hkv=2, N=64, d=64, scale=0.125, causal=0, dtype=0)
+        args.update(kw)
+        lib = fa.load()
+        return lib.fa_fwd(ptr(args["q"]), ptr(args["k"]), ptr(args["v"]), ptr(args["o"]), ptr(args["lse"]),
+                          args["B"], args["Hq"], args["Hkv"], args["N"], args["d"], args["scale"], args["causal"],
+                          args["dtype"], ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+    assert call(N=-1) == fa.FA_ERR_INVALID
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(Hq=3, Hkv=2) == fa.FA_ERR_INVALID
+    assert call(q=None) == fa.FA_ERR_INVALID
+    assert call(causal=2) == fa.FA_ERR_INVALID
+    assert call(dtype=7) == fa.FA_ERR_INVALID
+    assert call(scale=float("nan")) == fa.FA_ERR_INVALID
+    qm = torch.empty(q.numel() + 8, dtype=torch.bfloat16, device="cuda")[1:1 + q.numel()].view(q.shape)
+    assert call(q=qm) == fa.FA_ERR_INVALID  # 2-byte aligned pointer
+    assert call(B=0) == fa.FA_OK and call(N=0) == fa.FA_OK  # empty problems: nothing to do
+    torch.cuda.synchronize()
+    assert torch.all(o == 7.0) and torch.all(lse == 7.0)
+    # backward: unsupported dtype/d and a short workspace
+    do = torch.randn_like(q)
+    dq, dk, dv = (torch.full_like(q, 3.0) for _ in range(3))
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fa.FAError) as e:
+        fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, small, False, 0.125)
+    assert e.value.status == fa.FA_ERR_WORKSPACE
+    q256 = torch.zeros(1, 1, 8, 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fa.FAError) as e:
+        fa.backward(q256, q256, q256, q256, torch.zeros(1, 1, 8, device="cuda"), q256)
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert torch.all(dq == 3.0) and torch.all(dk == 3.0) and torch.all(dv == 3.0)
+
+
+def test_bounded_wait_timeout_reports_status(fa):
+    assert fa.fa_last_device_status() == fa.FA_OK
+    assert fa.fa_selftest_wait_timeout(50_000_000) == fa.FA_OK  # 50 ms
+    assert fa.fa_last_device_status() == fa.FA_ERR_TIMEOUT
+    assert fa.fa_last_device_status() == fa.FA_OK  # cleared by the read
+    # the context is still usable afterwards
+    inp = INP.make_inputs(1, 1, 1, 130, 64, "bf16", seed=2)
+    o, lse = _run_fwd(fa, inp, True, 0.125)
+    ro, rl = ORACLE.attention_forward(*(INP.as_f64(inp[n]) for n in "qkv"), 0.125, True)
+    assert np.max(np.abs(INP.as_f64(o) - ro)) <= O_TOL_BF16
