@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""Throughput of exact causal attention, forward + backward, bf16, on B200.
+
+One step is the whole hot path over one batch: ``fa_fwd`` (O, LSE), then the
+three backward stages ``fa_bwd_prep`` (D, padded LSE, zeroed dQ accumulator),
+``fa_bwd_main`` (recompute, dK, dV, dQ accumulation) and ``fa_bwd_dq``
+(dQ to bf16), on B=2, Hq=Hkv=32, N=8192, d=128, causal, synthetic N(0,1)
+inputs rounded to bf16. FLOPs follow the usual convention: forward
+4*B*Hq*N^2*d, halved when causal; backward 2.5 times the forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0. ``value`` is the whole-job TFLOP/s with
+inputs resident in HBM (max over ranks of the device time); ``e2e`` is the
+same metric measured through the C ABI with pinned host buffers, including
+the host-to-device copies of Q, K, V, dO and the device-to-host copies of O,
+LSE, dQ, dK, dV. ``--impl reference`` times the fp64 CPU oracle on a bounded
+sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd / fwd+bwd TFLOP/s, bf16 causal N=8k d=128, % of B200 BF16 peak"
+SHAPE = dict(B=2, Hq=32, Hkv=32, N=8192, d=128)
+CAUSAL = True
+SEED = 1003
+WORKLOAD_NAME = "causal bf16 attention forward+backward, B=2 Hq=32 Hkv=32 N=8192 d=128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# Measured DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+# of the dominant kernel, with the hash of the kernel source it was taken on.
+# Reported only while the source still hashes to the same value.
+TRAFFIC = {}
+
+
+def fwd_flops(B, Hq, N, d, causal):
+    f = 4.0 * B * Hq * N * N * d
+    return f / 2 if causal else f
+
+
+def bwd_flops(B, Hq, N, d, causal):
+    return 2.5 * fwd_flops(B, Hq, N, d, causal)
+
+
+def algorithmic_bytes(B, Hq, Hkv, N, d):
+    """Bytes each kernel must move at least once (bf16 tensors, f32 LSE/D/accumulator)."""
+    q = B * Hq * N * d * 2
+    kv = B * Hkv * N * d * 2
+    rows = B * Hq * N * 4
+    return {
+        "fwd": q + 2 * kv + q + rows,                     # read Q, K, V; write O, LSE
+        "bwd_prep": 2 * q + rows + 2 * rows + 2 * q,      # read O, dO, LSE; write D, LSE2, zero dQacc (f32)
+        "bwd_main": 2 * q + 2 * kv + 2 * rows + 2 * kv + 2 * q * 2,  # read Q,dO,K,V,LSE2,D; write dK,dV; dQacc add
+        "bwd_dq": 2 * q + q,                              # read dQacc (f32), write dQ
+    }
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_61_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            data = json.load(f)
+        return data, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons with nvidia-smi while running."""
+
+    def __init__(self, gpu_index: str):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_index, f"--query-gpu={CLOCK_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) != 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        max_power = max(r[2] for r in rows)
+        loaded = [r for r in rows if r[2] >= 0.5 * max_power] or rows
+        reasons = sorted({REASON_NAMES[i] for r in loaded for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max_power}
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def oracle_sample(inp_np, block: int, scale: float):
+    """Run the fp64 oracle forward + backward on one sampled block of query rows.
+
+    Block ``block`` picks head ``block % (B*Hq)`` and the 512 query rows
+    ``r0, r0+16, ...`` (every 16th row, so the rows see keys spread over the
+    causal range). Returns the algorithmic FLOPs of that sample under the
+    same convention as the GPU numbers (only visible keys counted).
+    """
+    import oracle.attention as ref  # test infrastructure: CPU-baseline leg only
+
+    B, Hq, N, d = inp_np["q"].shape
+    bh = block % (B * Hq)
+    b, h = divmod(bh, Hq)
+    rows = list(range(block % 16, N, 16))
+    q, k, v, do = (inp_np[n] for n in ("q", "k", "v", "do"))
+    ref.attention_forward_rows(q, k, v, scale, CAUSAL, b, h, rows)
+    ref.attention_backward_rows(q, k, v, do, scale, CAUSAL, b, h, rows)
+    visible = sum((r + 1) if CAUSAL else N for r in rows)
+    return 4.0 * d * visible * 3.5
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def sample_inputs_numpy():
+    """The benchmark workload's inputs in float64 (exact upcast of the bf16 values)."""
+    from exact_io_aware_61_b200 import inputs as inp_mod
+
+    inp = inp_mod.make_inputs(SHAPE["B"], SHAPE["Hq"], SHAPE["Hkv"], SHAPE["N"], SHAPE["d"], "bf16", SEED, grad=True)
+    return {n: inp_mod.as_f64(t) for n, t in inp.items()}
+
+
+def cpu_baseline(min_seconds=10.0, max_seconds=30.0):
+    inp = sample_inputs_numpy()
+    scale = SHAPE["d"] ** -0.5
+    flops, blocks = 0.0, 0
+    t0 = time.perf_counter()
+    while True:
+        flops += oracle_sample(inp, blocks, scale)
+        blocks += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or el + el / blocks > max_seconds:
+            break
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{blocks} blocks of 512 query rows (every 16th row of one head), fp64 numpy forward + "
+                      f"backward of the full workload's inputs, {el:.1f} s"}
+
+
+# ----------------------------------------------------------------- helpers
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest ``value`` over all ranks (identity for one rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+
+        t = torch.zeros(1, device=device)
+        dist.all_reduce(t)
+
+
+def physical_gpu_index(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# -------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local):
+    import torch
+
+    import exact_io_aware_61_b200 as fa
+    from exact_io_aware_61_b200 import inputs as inp_mod
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    fa.load()
+    B, Hq, Hkv, N, d = (SHAPE[k] for k in ("B", "Hq", "Hkv", "N", "d"))
+    scale = d ** -0.5
+    host = inp_mod.make_inputs(B, Hq, Hkv, N, d, "bf16", SEED + rank, grad=True)
+    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, Hq, Hkv, N, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fa.fa_fwd(q, k, v, o, lse, CAUSAL, scale, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        fa.fa_bwd_prep(o, lse, do, ws, Hkv, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        fa.fa_bwd_main(q, k, v, do, dk, dv, ws, CAUSAL, scale, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        fa.fa_bwd_dq(dq, ws, Hkv, stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.fa_last_device_status(stream) != fa.FA_OK:
+        raise RuntimeError("device status reports a timeout during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(physical_gpu_index(local))
+    sampler.start()
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(events[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    status = fa.fa_last_device_status(stream)
+    if status != fa.FA_OK:
+        raise RuntimeError(f"device status {fa.status_string(status)} in the timed region")
+
+    elapsed_ms = start.elapsed_time(end)
+    per_kernel = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in events)
+                  for i, name in enumerate(("fwd", "bwd_prep", "bwd_main", "bwd_dq"))}
+    max_ms = max_over_ranks(elapsed_ms, world, dev)
+
+    f_fwd = fwd_flops(B, Hq, N, d, CAUSAL)
+    f_bwd = bwd_flops(B, Hq, N, d, CAUSAL)
+    step_flops = f_fwd + f_bwd
+    value = world * step_flops * args.steps / (max_ms / 1e3) / 1e12
+    bwd_ms = per_kernel["bwd_prep"] + per_kernel["bwd_main"] + per_kernel["bwd_dq"]
+
+    # end to end through the C ABI: pinned host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hq_, hk_, hv_, hdo_ = (host[n].pin_memory() for n in ("q", "k", "v", "do"))
+        outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
+        e2e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            for dst, src in ((q, hq_), (k, hk_), (v, hv_), (do, hdo_)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in zip(outs, (o, lse, dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1), world, dev)
+        h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_, hdo_))
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        e2e = {"value": world * step_flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "ms_per_step": e2e_ms / e2e_steps}
+
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    peak_tf = float(peaks["bf16_tflops"])
+    hbm = float(peaks["hbm_gbs"])
+    nbytes = algorithmic_bytes(B, Hq, Hkv, N, d)
+    kernels = {
+        "fwd": {"ms": per_kernel["fwd"], "tflops": f_fwd / per_kernel["fwd"] / 1e9,
+                "gbs": nbytes["fwd"] / per_kernel["fwd"] / 1e6},
+        "bwd_main": {"ms": per_kernel["bwd_main"], "tflops": f_bwd / per_kernel["bwd_main"] / 1e9,
+                     "gbs": nbytes["bwd_main"] / per_kernel["bwd_main"] / 1e6},
+        "bwd_prep": {"ms": per_kernel["bwd_prep"], "gbs": nbytes["bwd_prep"] / per_kernel["bwd_prep"] / 1e6},
+        "bwd_dq": {"ms": per_kernel["bwd_dq"], "gbs": nbytes["bwd_dq"] / per_kernel["bwd_dq"] / 1e6},
+    }
+    dominant = "bwd_main" if per_kernel["bwd_main"] >= per_kernel["fwd"] else "fwd"
+    dom_flops = f_bwd if dominant == "bwd_main" else f_fwd
+    achieved = dom_flops / per_kernel[dominant] / 1e9
+    src_hash = kernel_source_hash()
+    traffic = TRAFFIC.get(dominant)
+    traffic_val = traffic["bytes"] if traffic and traffic.get("src") == src_hash else None
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: i.i.d. N(0,1) rounded to bf16, seeded",
+        "config": {"workload": WORKLOAD_NAME, "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": CAUSAL,
+                   "parallelism": f"{world} independent replicas (one per GPU), no collective",
+                   "l2": "no flush: every step streams > 1 GB and each of Q, K, V, O, dO is 134 MB (> 126 MB L2)"},
+        "fwd_tflops": round(f_fwd / per_kernel["fwd"] / 1e9, 2),
+        "bwd_tflops": round(f_bwd / bwd_ms / 1e9, 2),
+        "pct_of_peak": {"fwd": round(100 * f_fwd / per_kernel["fwd"] / 1e9 / peak_tf, 2),
+                        "bwd": round(100 * f_bwd / bwd_ms / 1e9 / peak_tf, 2),
+                        "step": round(100 * value / world / peak_tf, 2),
+                        "peak_tflops": peak_tf, "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "kernels": {k: {kk: round(vv, 4) for kk, vv in v.items()} for k, v in kernels.items()},
+        "roofline": {"kernel": "fa_bwd_main_kernel<128>" if dominant == "bwd_main" else "fa_fwd_bf16_kernel<128>",
+                     "bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_tf, 4), "traffic": traffic_val,
+                     "algorithmic_bytes": nbytes[dominant],
+                     "peak_note": f"{peak_src} (burst bf16 GEMM)", "hbm_peak_gbs": hbm},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+        "kernel_src": src_hash,
+    }
+    if e2e is not None:
+        out["e2e"] = {k: (round(v, 4) if isinstance(v, float) else v) for k, v in e2e.items()}
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(out), flush=True)
+
+
+# --------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return  # rank 0 alone times the oracle; the others exit without work
+    inp = sample_inputs_numpy()
+    scale = SHAPE["d"] ** -0.5
+    for i in range(args.warmup):
+        oracle_sample(inp, i, scale)
+    flops = 0.0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        flops += oracle_sample(inp, args.warmup + i, scale)
+    el = time.perf_counter() - t0
+    value = flops / el / 1e12
+    cores = blas_threads()
+    out = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic: i.i.d. N(0,1) rounded to bf16, seeded",
+        "config": {"workload": WORKLOAD_NAME, **SHAPE, "causal": CAUSAL,
+                   "parallelism": "rank 0 only, host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "per step: 512 query rows (every 16th row of one head), fp64 numpy forward "
+                                   "+ backward"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error(f"--gpus {args.gpus} needs a launch with torch.distributed.run (one rank per GPU)")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -19,6 +19,9 @@ from ._lib import (  # noqa: F401
     FAError,
     backward,
     fa_bwd,
+    fa_bwd_dq,
+    fa_bwd_main,
+    fa_bwd_prep,
     fa_bwd_workspace_size,
     fa_fwd,
     fa_last_device_status,

@@ -23,6 +23,9 @@ FA_BF16, FA_F32 = 0, 1
 EXPORTED = (
     "fa_fwd",
     "fa_bwd",
+    "fa_bwd_prep",
+    "fa_bwd_main",
+    "fa_bwd_dq",
     "fa_bwd_workspace_size",
     "fa_status_string",
     "fa_last_device_status",
@@ -56,6 +59,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_fwd.restype = i
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp]
         lib.fa_bwd.restype = i
+        lib.fa_bwd_prep.argtypes = [vp, vp, vp, vp, sz, i, i, i, i, i, i, vp]
+        lib.fa_bwd_prep.restype = i
+        lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp]
+        lib.fa_bwd_main.restype = i
+        lib.fa_bwd_dq.argtypes = [vp, vp, sz, i, i, i, i, i, i, vp]
+        lib.fa_bwd_dq.restype = i
         lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i]
         lib.fa_bwd_workspace_size.restype = sz
         lib.fa_status_string.argtypes = [i]
@@ -131,6 +140,43 @@ def fa_bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool, scale: floa
                        ctypes.c_void_p(_stream_ptr(stream)))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd")
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    return ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size()
+
+
+def fa_bwd_prep(o, lse, do, workspace, Hkv: int, stream=None) -> None:
+    """Stage 1 of ``fa_bwd``: D, padded log2 LSE and a zeroed dQ accumulator in ``workspace``."""
+    B, Hq, N, d = o.shape
+    ws, nbytes = _ws(workspace)
+    rc = load().fa_bwd_prep(_ptr(o), _ptr(lse), _ptr(do), ws, nbytes, B, Hq, Hkv, N, d, _dtype_code(o),
+                            ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_prep")
+
+
+def fa_bwd_main(q, k, v, do, dk, dv, workspace, causal: bool, scale: float, stream=None) -> None:
+    """Stage 2 of ``fa_bwd``: the recompute kernel (dK, dV, and dQ into the accumulator)."""
+    B, Hq, N, d = q.shape
+    ws, nbytes = _ws(workspace)
+    rc = load().fa_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk), _ptr(dv), ws, nbytes, B, Hq,
+                            k.shape[1], N, d, float(scale), int(bool(causal)), _dtype_code(q),
+                            ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_main")
+
+
+def fa_bwd_dq(dq, workspace, Hkv: int, stream=None) -> None:
+    """Stage 3 of ``fa_bwd``: f32 accumulator -> bf16 ``dq``."""
+    B, Hq, N, d = dq.shape
+    ws, nbytes = _ws(workspace)
+    rc = load().fa_bwd_dq(_ptr(dq), ws, nbytes, B, Hq, Hkv, N, d, _dtype_code(dq),
+                          ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_dq")
 
 
 def forward(q, k, v, causal: bool = False, scale: float | None = None, stream=None):

@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <initializer_list>
 #include <mutex>
 
 #include <cuda.h>
@@ -172,45 +173,60 @@ int launch_fwd_f32(const void* q, const void* k, const void* v, void* o, float* 
 
 size_t padded_rows(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 
-template <int HD>
-int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-               void* dq, void* dk, void* dv, void* ws, int B, int Hq, int Hkv, int N, float scale, int causal,
-               cudaStream_t stream) {
-  using C = fa::BwdCfg<HD>;
+// Workspace carve-up: D [B*Hq][Npad], LSE*log2(e) [B*Hq][Npad], dQ accumulator [B*Hq][N][d], all f32.
+struct BwdWorkspace {
+  float* delta;
+  float* lse2;
+  float* dq_acc;
+};
+
+BwdWorkspace carve(void* ws, int B, int Hq, int N) {
   const size_t npad = padded_rows(N);
   const size_t rows_q = static_cast<size_t>(B) * Hq;
-  float* ws_delta = static_cast<float*>(ws);
-  float* ws_lse2 = ws_delta + rows_q * npad;
-  float* dq_acc = ws_lse2 + rows_q * npad;
+  BwdWorkspace w;
+  w.delta = static_cast<float*>(ws);
+  w.lse2 = w.delta + rows_q * npad;
+  w.dq_acc = w.lse2 + rows_q * npad;
+  return w;
+}
 
+template <int HD>
+int launch_bwd_prep(const void* o, const float* lse, const void* dO, void* ws, int B, int Hq, int N,
+                    cudaStream_t stream) {
+  const BwdWorkspace w = carve(ws, B, Hq, N);
+  const size_t npad = padded_rows(N);
   fa::BwdPrepParams pp;
   pp.o = static_cast<const __nv_bfloat16*>(o);
   pp.dO = static_cast<const __nv_bfloat16*>(dO);
   pp.lse = lse;
-  pp.ws_delta = ws_delta;
-  pp.ws_lse2 = ws_lse2;
-  pp.dq_acc = dq_acc;
+  pp.ws_delta = w.delta;
+  pp.ws_lse2 = w.lse2;
+  pp.dq_acc = w.dq_acc;
   pp.N = N;
   pp.Npad = static_cast<int>(npad);
-  const long long prep_blocks = static_cast<long long>(npad / 32) * static_cast<long long>(rows_q);
-  if (prep_blocks > INT32_MAX) return FA_ERR_INVALID;
-  fa::fa_bwd_prep_kernel<HD><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(pp);
-  int rc = launch_status();
-  if (rc != FA_OK) return rc;
+  const long long blocks = static_cast<long long>(npad / 32) * B * Hq;
+  if (blocks > INT32_MAX) return FA_ERR_INVALID;
+  fa::fa_bwd_prep_kernel<HD><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(pp);
+  return launch_status();
+}
 
+template <int HD>
+int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* ws,
+                    int B, int Hq, int Hkv, int N, float scale, int causal, cudaStream_t stream) {
+  using C = fa::BwdCfg<HD>;
+  const BwdWorkspace w = carve(ws, B, Hq, N);
+  const size_t npad = padded_rows(N);
+  const uint64_t rows_q = static_cast<uint64_t>(B) * Hq, rows_kv = static_cast<uint64_t>(B) * Hkv;
   CUtensorMap mq, mk, mv, mdo, mdq;
-  rc = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
-  if (rc == FA_OK)
-    rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
-  if (rc == FA_OK)
-    rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  int rc = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
+  if (rc == FA_OK) rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
+  if (rc == FA_OK) rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
   if (rc == FA_OK) rc = make_map(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
-  if (rc == FA_OK) rc = make_map(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, N, rows_q, 32, 128);
+  if (rc == FA_OK) rc = make_map(&mdq, w.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, N, rows_q, 32, 128);
   if (rc != FA_OK) return rc;
-
   fa::BwdParams p;
-  p.ws_delta = ws_delta;
-  p.ws_lse2 = ws_lse2;
+  p.ws_delta = w.delta;
+  p.ws_lse2 = w.lse2;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.N = N;
@@ -226,14 +242,31 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   if (blocks > INT32_MAX) return FA_ERR_INVALID;
   fa::fa_bwd_main_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
                                                                                                     mdq, p);
-  rc = launch_status();
-  if (rc != FA_OK) return rc;
+  return launch_status();
+}
 
-  const size_t n4 = rows_q * static_cast<size_t>(N) * HD / 4;
+int launch_bwd_dq(void* dq, void* ws, int B, int Hq, int N, int d, cudaStream_t stream) {
+  const BwdWorkspace w = carve(ws, B, Hq, N);
+  const size_t n4 = static_cast<size_t>(B) * Hq * static_cast<size_t>(N) * d / 4;
   const size_t want = (n4 + 255) / 256;
   const unsigned grid = static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
-  fa::fa_bwd_dq_kernel<<<grid, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n4);
+  fa::fa_bwd_dq_kernel<<<grid, 256, 0, stream>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), n4);
   return launch_status();
+}
+
+// Checks shared by the backward entry points. `ptrs` must all be 16-byte aligned and non-null.
+int check_bwd(std::initializer_list<const void*> ptrs, void* workspace, size_t workspace_bytes, int B, int Hq,
+              int Hkv, int N, int d, float scale, int causal, int dtype, int* dev) {
+  int rc = check_shape(B, Hq, Hkv, N, d, scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return -1;  // empty: nothing to launch
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return FA_ERR_INVALID;
+  if (workspace == nullptr || workspace_bytes < fa_bwd_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_INVALID;
+  if ((rc = check_device(dev)) != FA_OK) return rc;
+  return prepare_kernels(*dev);
 }
 
 }  // namespace
@@ -286,24 +319,53 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
   return sizeof(float) * (2 * rows_q * padded_rows(N) + rows_q * static_cast<size_t>(N) * d);
 }
 
+int fa_bwd_prep(const void* o, const float* lse, const void* dO, void* workspace, size_t workspace_bytes, int B,
+                int Hq, int Hkv, int N, int d, int dtype, fa_stream_t stream) {
+  int dev = 0;
+  int rc = check_bwd({o, lse, dO}, workspace, workspace_bytes, B, Hq, Hkv, N, d, 1.0f, 0, dtype, &dev);
+  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd_prep<64>(o, lse, dO, workspace, B, Hq, N, s)
+                 : launch_bwd_prep<128>(o, lse, dO, workspace, B, Hq, N, s);
+}
+
+int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* workspace,
+                size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale, int causal, int dtype,
+                fa_stream_t stream) {
+  int dev = 0;
+  int rc = check_bwd({q, k, v, dO, dk, dv}, workspace, workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype, &dev);
+  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd_main<64>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s)
+                 : launch_bwd_main<128>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s);
+}
+
+int fa_bwd_dq(void* dq, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int dtype,
+              fa_stream_t stream) {
+  int dev = 0;
+  int rc = check_bwd({dq}, workspace, workspace_bytes, B, Hq, Hkv, N, d, 1.0f, 0, dtype, &dev);
+  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
+  return launch_bwd_dq(dq, workspace, B, Hq, N, d, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
            void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
            float scale, int causal, int dtype, fa_stream_t stream) {
-  int rc = check_shape(B, Hq, Hkv, N, d, scale, causal, dtype);
-  if (rc != FA_OK) return rc;
-  if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
-  if (B == 0 || N == 0) return FA_OK;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_INVALID;
-  if (workspace == nullptr || workspace_bytes < fa_bwd_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return FA_ERR_INVALID;
   int dev = 0;
-  if ((rc = check_device(&dev)) != FA_OK) return rc;
-  if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
+  int rc = check_bwd({q, k, v, o, lse, dO, dq, dk, dv}, workspace, workspace_bytes, B, Hq, Hkv, N, d, scale, causal,
+                     dtype, &dev);
+  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_bwd<64>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s);
-  return launch_bwd<128>(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s);
+  if (d == 64) {
+    if ((rc = launch_bwd_prep<64>(o, lse, dO, workspace, B, Hq, N, s)) != FA_OK) return rc;
+    if ((rc = launch_bwd_main<64>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
+      return rc;
+  } else {
+    if ((rc = launch_bwd_prep<128>(o, lse, dO, workspace, B, Hq, N, s)) != FA_OK) return rc;
+    if ((rc = launch_bwd_main<128>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
+      return rc;
+  }
+  return launch_bwd_dq(dq, workspace, B, Hq, N, d, s);
 }
 
 int fa_last_device_status(fa_stream_t stream) {

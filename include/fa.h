@@ -130,6 +130,34 @@ FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o,
            int B, int Hq, int Hkv, int N, int d, float scale, int causal,
            int dtype, fa_stream_t stream);
 
+/*
+ * The three stages of fa_bwd as separate calls, for callers that want to
+ * time or schedule them one by one. Calling them in this order on one
+ * stream, with the same sizes and workspace, is exactly fa_bwd. Arguments
+ * mean what they mean for fa_bwd; the same checks and error codes apply.
+ *
+ * fa_bwd_prep -- writes D = rowsum(dO * O) and LSE * log2(e) into the
+ *   workspace (128-row padded per head; padding rows get D = 0 and an
+ *   infinite LSE, i.e. zero weight) and zeroes the f32 dQ accumulator.
+ *   Reads o, lse, dO.
+ * fa_bwd_main -- the recompute kernel: per 128-key tile of each KV head it
+ *   rebuilds P from Q, K and the padded LSE, and forms dV, dP, dS, dK (written
+ *   to dk, dv) and adds each dQ tile into the accumulator. Needs fa_bwd_prep
+ *   to have run on the same workspace.
+ * fa_bwd_dq -- converts the f32 dQ accumulator to dq (bf16).
+ */
+FA_API int fa_bwd_prep(const void* o, const float* lse, const void* dO,
+                void* workspace, size_t workspace_bytes,
+                int B, int Hq, int Hkv, int N, int d, int dtype,
+                fa_stream_t stream);
+FA_API int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO,
+                void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                int dtype, fa_stream_t stream);
+FA_API int fa_bwd_dq(void* dq, void* workspace, size_t workspace_bytes,
+              int B, int Hq, int Hkv, int N, int d, int dtype,
+              fa_stream_t stream);
+
 /* Human-readable name of a fa_status value (static string, never NULL). */
 FA_API const char* fa_status_string(int status);
 

@@ -58,6 +58,7 @@ __all__ = [
     "attention_forward_rows",
     "online_softmax_forward",
     "attention_backward",
+    "attention_backward_rows",
     "score_matrix_bytes",
 ]
 
@@ -245,6 +246,32 @@ def attention_backward(q, k, v, do, scale: float, causal: bool):
             dq[b, h] = scale * (ds @ k[b, hk])
             dk[b, hk] += scale * (ds.T @ q[b, h])
     return dq, dk, dv, D
+
+
+def attention_backward_rows(q, k, v, do, scale: float, causal: bool, b: int, h: int, rows):
+    """The backward restricted to the query positions ``rows`` of one (batch, head).
+
+    Same formulas as :func:`attention_backward`. Returns ``(dQ_rows, dK_part,
+    dV_part)``: the dQ rows of those queries and the share of dK and dV (of
+    the KV head ``h`` reads) that those queries contribute. Summing the shares
+    over a partition of all rows and heads of a group gives dK and dV.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    Hq = np.shape(q)[1]
+    Hkv = np.shape(k)[1]
+    hk = kv_head_of(h, Hq, Hkv)
+    q_rows = _f64(np.asarray(q)[b, h][rows])
+    do_rows = _f64(np.asarray(do)[b, h][rows])
+    k_bh = _f64(np.asarray(k)[b, hk])
+    v_bh = _f64(np.asarray(v)[b, hk])
+    s = masked_scores(q_rows, k_bh, scale, causal, rows=rows)
+    p = softmax_rows(s)[0]
+    o_rows = p @ v_bh
+    dv_part = p.T @ do_rows
+    dp = do_rows @ v_bh.T
+    D = np.sum(do_rows * o_rows, axis=1)
+    ds = score_gradient(p, dp, D)
+    return scale * (ds @ k_bh), scale * (ds.T @ q_rows), dv_part
 
 
 def score_gradient(p, dp, D):

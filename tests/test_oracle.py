@@ -256,7 +256,28 @@ def check_rows_helper_matches_full(o):
         assert np.max(np.abs(rl - full_l[1, 3, rows])) < 1e-14
 
 
+def check_backward_rows_partition(o):
+    # The row-restricted backward: its dQ rows are the full dQ rows, and its
+    # dK/dV shares summed over a partition of all query rows (and the heads of
+    # each group) give the full dK/dV.
+    q, k, v = _qkv(B=1, Hq=4, Hkv=2, N=21, d=3, seed=61)
+    do = _rand(q.shape, 67)
+    parts = [np.arange(0, 21, 3), np.arange(1, 21, 3), np.arange(2, 21, 3)]
+    for causal in (False, True):
+        dq, dk, dv, _ = o.attention_backward(q, k, v, do, 0.7, causal)
+        dk_sum, dv_sum = np.zeros_like(dk), np.zeros_like(dv)
+        for h in range(4):
+            for rows in parts:
+                rq, rk, rv = o.attention_backward_rows(q, k, v, do, 0.7, causal, 0, h, rows)
+                assert np.max(np.abs(rq - dq[0, h, rows])) < 1e-13
+                dk_sum[0, h // 2] += rk
+                dv_sum[0, h // 2] += rv
+        assert np.max(np.abs(dk_sum - dk)) < 1e-12
+        assert np.max(np.abs(dv_sum - dv)) < 1e-12
+
+
 ALL_CHECKS = [
+    check_backward_rows_partition,
     check_rows_sum_to_one,
     check_single_key_returns_value,
     check_zero_query_uniform,
