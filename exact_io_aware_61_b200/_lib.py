@@ -26,6 +26,7 @@ EXPORTED = (
     "fa_bwd_prep",
     "fa_bwd_main",
     "fa_bwd_dq",
+    "fa_bwd_noalloc",
     "fa_bwd_workspace_size",
     "fa_status_string",
     "fa_last_device_status",
@@ -65,6 +66,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_bwd_main.restype = i
         lib.fa_bwd_dq.argtypes = [vp, vp, sz, i, i, i, i, i, i, vp]
         lib.fa_bwd_dq.restype = i
+        lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+        lib.fa_bwd_noalloc.restype = i
         lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i]
         lib.fa_bwd_workspace_size.restype = sz
         lib.fa_status_string.argtypes = [i]
@@ -177,6 +180,29 @@ def fa_bwd_dq(dq, workspace, Hkv: int, stream=None) -> None:
                           ctypes.c_void_p(_stream_ptr(stream)))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd_dq")
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024  # FA_NOALLOC_SCRATCH_BYTES in include/fa.h
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, causal: bool, scale: float, stream=None) -> None:
+    """Call ``fa_bwd_noalloc``: the backward with the library's built-in scratch.
+
+    For callers that cannot allocate device memory (a locked or pre-planned
+    allocator, plain C callers without one). Problems needing more than
+    ``NOALLOC_SCRATCH_BYTES`` of scratch raise ``FAError`` (FA_ERR_WORKSPACE).
+    Calls share one scratch array per GPU: do not let two of them overlap on
+    the device.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse), ("do", do), ("dq", dq),
+                    ("dk", dk), ("dv", dv)):
+        _check_tensor(name, t, q.device)
+    B, Hq, N, d = q.shape
+    rc = load().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                               _ptr(dv), B, Hq, k.shape[1], N, d, float(scale), int(bool(causal)),
+                               _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_noalloc")
 
 
 def forward(q, k, v, causal: bool = False, scale: float | None = None, stream=None):

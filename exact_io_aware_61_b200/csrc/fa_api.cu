@@ -368,6 +368,75 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   return launch_bwd_dq(dq, workspace, B, Hq, N, d, s);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward without caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// backward: code inside a region where the allocator must not be touched
+// (a caching allocator that is locked, a pre-planned memory arena, a runtime
+// that forbids cudaMalloc after start-up), or plain C callers with no
+// allocator of their own. For them the scratch lives in a fixed array in
+// device memory that the library owns: every GPU that loads the library
+// holds it until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = FA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device with that device current. In host code the array's name is only
+// a host-side stand-in, never a device address.
+int noalloc_scratch(int dev, void** out) {
+  static std::mutex mu;
+  static void* addr[128] = {};
+  if (dev < 0 || dev >= 128) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                   void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                   int dtype, fa_stream_t stream) {
+  int rc = check_shape(B, Hq, Hkv, N, d, scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return FA_OK;
+  if (fa_bwd_workspace_size(B, Hq, Hkv, N, d) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  int dev = 0;
+  if ((rc = check_device(&dev)) != FA_OK) return rc;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(dev, &scratch)) != FA_OK) return rc;
+  rc = check_bwd({q, k, v, o, lse, dO, dq, dk, dv}, scratch, kNoAllocScratchBytes, B, Hq, Hkv, N, d, scale, causal,
+                 dtype, &dev);
+  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
+  // The prep kernel rewrites every scratch byte this problem reads (D, LSE,
+  // and the dQ accumulator, which it zeroes), so what an earlier call left
+  // in the array does not matter.
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) {
+    if ((rc = launch_bwd_prep<64>(o, lse, dO, scratch, B, Hq, N, s)) != FA_OK) return rc;
+    if ((rc = launch_bwd_main<64>(q, k, v, dO, dk, dv, scratch, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
+      return rc;
+  } else {
+    if ((rc = launch_bwd_prep<128>(o, lse, dO, scratch, B, Hq, N, s)) != FA_OK) return rc;
+    if ((rc = launch_bwd_main<128>(q, k, v, dO, dk, dv, scratch, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
+      return rc;
+  }
+  return launch_bwd_dq(dq, scratch, B, Hq, N, d, s);
+}
+
 int fa_last_device_status(fa_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;

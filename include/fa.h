@@ -158,6 +158,36 @@ FA_API int fa_bwd_dq(void* dq, void* workspace, size_t workspace_bytes,
               int B, int Hq, int Hkv, int N, int d, int dtype,
               fa_stream_t stream);
 
+/*
+ * fa_bwd_noalloc -- fa_bwd for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot hand fa_bwd a workspace: code running where the device allocator
+ * must not be touched (a locked caching allocator, a fixed memory arena
+ * planned ahead of time, a runtime that forbids cudaMalloc once it has
+ * started) and plain C callers with no allocator of their own.
+ *
+ * Same arguments, results and checks as fa_bwd, without workspace and
+ * workspace_bytes. The scratch is a fixed device array of
+ * FA_NOALLOC_SCRATCH_BYTES bytes inside the library, present on every GPU
+ * that loads the library until the process exits. Problems whose
+ * fa_bwd_workspace_size() exceeds it return FA_ERR_WORKSPACE without
+ * launching anything. The call allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls share the one array: the call rewrites every scratch
+ * byte it reads (it zeroes the dQ accumulator itself), but two calls whose
+ * kernels overlap on the GPU (different streams, no ordering between them)
+ * race on it and give wrong results. Order such calls on one stream.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+FA_API int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                   const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                   int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                   int dtype, fa_stream_t stream);
+
 /* Human-readable name of a fa_status value (static string, never NULL). */
 FA_API const char* fa_status_string(int status);
 
