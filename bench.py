@@ -466,7 +466,14 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default=None,
+                    help="B,Hq,Hkv,N,d of a smaller case for profiling (default: the benchmark workload)")
     args = ap.parse_args(argv)
+    if args.shape:
+        global WORKLOAD_NAME
+        B, Hq, Hkv, N, d = (int(x) for x in args.shape.split(","))
+        SHAPE.update(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d)
+        WORKLOAD_NAME = f"causal bf16 attention forward+backward, B={B} Hq={Hq} Hkv={Hkv} N={N} d={d}"
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_env()

@@ -4,6 +4,8 @@
 
 #include <atomic>
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <cstdint>
 #include <initializer_list>
 #include <mutex>
@@ -16,6 +18,7 @@
 #include "fa.h"
 #include "sm100_ptx.cuh"
 #include "fwd_sm100.cuh"
+#include "fwd2_sm100.cuh"
 #include "fwd_f32.cuh"
 #include "bwd_sm100.cuh"
 
@@ -75,8 +78,8 @@ int prepare_kernels(int dev) {
   auto set = [&](const void* fn, int bytes) {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   };
-  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<64>), fa::FwdCfg<64>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<128>), fa::FwdCfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<64>), fa::Fwd2Cfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<128>), fa::Fwd2Cfg<128>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<256>), fa::FwdCfg<256>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<64>), fa::fwd_f32_smem_bytes<64>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<128>), fa::fwd_f32_smem_bytes<128>());
@@ -122,18 +125,47 @@ int check_shape(int B, int Hq, int Hkv, int N, int d, float scale, int causal, i
 
 unsigned long long timeout_now() { return static_cast<unsigned long long>(g_timeout_ns.load()); }
 
-int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+bool verbose() {
+  static const bool v = [] {
+    const char* e = std::getenv("FA_VERBOSE");
+    return e != nullptr && e[0] != '\0' && e[0] != '0';
+  }();
+  return v;
+}
+
+// Status of the launch just made; with FA_VERBOSE set, a failure is described
+// on stderr together with the kernel's resource attributes.
+int launch_status(const void* kernel = nullptr) {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return FA_OK;
+  if (verbose()) {
+    std::fprintf(stderr, "fa: launch failed: %s\n", cudaGetErrorString(e));
+    cudaFuncAttributes a;
+    if (kernel != nullptr && cudaFuncGetAttributes(&a, kernel) == cudaSuccess)
+      std::fprintf(stderr, "fa: kernel regs=%d maxThreads=%d staticSmem=%zu maxDynSmem=%d localBytes=%zu\n",
+                   a.numRegs, a.maxThreadsPerBlock, a.sharedSizeBytes, a.maxDynamicSharedSizeBytes,
+                   a.localSizeBytes);
+  }
+  return FA_ERR_CUDA;
+}
 
 template <int HD>
-int launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                    int N, float scale, int causal, cudaStream_t stream) {
-  using C = fa::FwdCfg<HD>;
+int make_qkv_maps(CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv, const void* q, const void* k, const void* v,
+                  int B, int Hq, int Hkv, int N) {
+  int rc = make_map(mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hq, 64, 128);
+  if (rc == FA_OK)
+    rc = make_map(mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  if (rc == FA_OK)
+    rc = make_map(mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  return rc;
+}
+
+// d = 256: one 128-row query tile per CTA (S double-buffered in TMEM).
+int launch_fwd_bf16_d256(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int N, float scale, int causal, cudaStream_t stream) {
+  using C = fa::FwdCfg<256>;
   CUtensorMap mq, mk, mv;
-  int rc = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hq, 64, 128);
-  if (rc == FA_OK)
-    rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
-  if (rc == FA_OK)
-    rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  int rc = make_qkv_maps<256>(&mq, &mk, &mv, q, k, v, B, Hq, Hkv, N);
   if (rc != FA_OK) return rc;
   fa::FwdParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -147,8 +179,46 @@ int launch_fwd_bf16(const void* q, const void* k, const void* v, void* o, float*
   p.timeout_ns = timeout_now();
   const long long blocks = static_cast<long long>(p.num_q_tiles) * B * Hq;
   if (blocks > INT32_MAX) return FA_ERR_INVALID;
-  fa::fa_fwd_bf16_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  fa::fa_fwd_bf16_kernel<256><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return launch_status();
+}
+
+// d = 64, 128: two 128-row query tiles per CTA.
+template <int HD>
+int launch_fwd_bf16_2tile(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int N, float scale, int causal, cudaStream_t stream) {
+  using C = fa::Fwd2Cfg<HD>;
+  CUtensorMap mq, mk, mv;
+  int rc = make_qkv_maps<HD>(&mq, &mk, &mv, q, k, v, B, Hq, Hkv, N);
+  if (rc != FA_OK) return rc;
+  fa::Fwd2Params p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.BH = B * Hq;
+  p.num_pairs = (N + 2 * C::BM - 1) / (2 * C::BM);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.timeout_ns = timeout_now();
+  const long long blocks = static_cast<long long>(p.num_pairs) * B * Hq;
+  if (blocks > INT32_MAX) return FA_ERR_INVALID;
+  // The kernel redistributes registers between its warpgroups (setmaxnreg);
+  // the split adds up to exactly LAUNCH_REGS per thread, so refuse to launch
+  // a build whose register count differs rather than risk a wait that never
+  // ends.
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<HD>)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (attr.numRegs != C::LAUNCH_REGS) {
+    if (verbose()) std::fprintf(stderr, "fa: 2-tile forward built with %d registers, expected %d\n", attr.numRegs,
+                                C::LAUNCH_REGS);
+    return FA_ERR_UNSUPPORTED;
+  }
+  fa::fa_fwd_bf16_2tile_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv,
+                                                                                                          p);
+  return launch_status(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<HD>));
 }
 
 template <int HD>
@@ -301,9 +371,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == FA_BF16) {
     switch (d) {
-      case 64: return launch_fwd_bf16<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
-      case 128: return launch_fwd_bf16<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
-      default: return launch_fwd_bf16<256>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
+      case 64: return launch_fwd_bf16_2tile<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
+      case 128: return launch_fwd_bf16_2tile<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
+      default: return launch_fwd_bf16_d256(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
     }
   }
   switch (d) {

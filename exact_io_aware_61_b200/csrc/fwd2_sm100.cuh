@@ -1,0 +1,416 @@
+// fwd2_sm100.cuh -- bf16 attention forward with two query tiles per CTA
+// (head dimensions 64 and 128).
+//
+// Same method as fwd_sm100.cuh (tiled pass, online softmax with a lazy
+// rescale of the running output, O = o / l once at the end), arranged so the
+// tensor core is never idle waiting on one softmax:
+//   * a CTA owns 256 query rows = two 128-row tiles of one (batch, head);
+//     both tiles read the same K/V tiles, halving shared-memory fills per
+//     FLOP;
+//   * each tile has its own softmax warpgroup and its own S and O in TMEM
+//     (S0 | S1 | O0 | O1 = 512 columns at d = 128), and the MMA issuer
+//     alternates PV0(j), S0(j+1), PV1(j), S1(j+1), so one warpgroup's
+//     softmax runs while the other tile's MMAs execute;
+//   * the softmax reads a whole 128-column score row with one TMEM load and
+//     reduces it with short trees (three-input max, packed f32x2 FMA/add).
+// Warps: 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA producer, 9 TMEM
+// allocator and MMA issuer, 10-11 idle. The block launches with 168
+// registers per thread; the two softmax warpgroups then take 216 each and the
+// third warpgroup keeps 72 (128 x (216 + 216 + 72) = 384 x 168). The host
+// launches the kernel only if its register count is exactly 168, since a
+// split above the launch allocation would wait forever.
+#pragma once
+
+#include <cuda.h>
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+template <int HD>
+struct Fwd2Cfg {
+  static constexpr int BM = 128;  // rows per query tile
+  static constexpr int BN = 128;  // keys per key tile
+  static constexpr int STAGES = HD == 64 ? 4 : 2;
+  static constexpr int Q_TILE_BYTES = BM * HD * 2;
+  static constexpr int KV_BYTES = BN * HD * 2;
+  static constexpr int SMEM_BYTES = 1024 + 2 * Q_TILE_BYTES + 2 * STAGES * KV_BYTES;
+  static constexpr int THREADS = 384;
+  static constexpr int LAUNCH_REGS = 168;  // the split below assumes exactly this
+  static constexpr int SOFTMAX_REGS = 216;
+  static constexpr int OTHER_REGS = 72;
+  static_assert(128 * (2 * SOFTMAX_REGS + OTHER_REGS) <= THREADS * LAUNCH_REGS, "register split exceeds launch");
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t TMEM_O = 256;  // O0 at 256, O1 at 256 + HD
+  static constexpr float RESCALE_THRESHOLD = 8.0f;
+  static constexpr int HEAD_GROUP = 8;  // heads scheduled together (K/V stay in L2)
+};
+
+struct Fwd2Params {
+  __nv_bfloat16* o;
+  float* lse;
+  int N, Hq, Hkv, BH, num_pairs;
+  float scale_log2;
+  int causal;
+  unsigned long long timeout_ns;
+};
+
+// ---------------------------------------------------------------- helpers
+
+FA_DEV float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+FA_DEV uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+FA_DEV void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+FA_DEV uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+FA_DEV uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+FA_DEV uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// One 32-lane x 128-column TMEM load (one column per register), waited.
+FA_DEV void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, "
+      "%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
+      "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, "
+      "%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, "
+      "%112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]),
+        "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]),
+        "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]),
+        "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]),
+        "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]),
+        "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]),
+        "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]),
+        "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]),
+        "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]),
+        "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr)
+      : "memory");
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int HD>
+// 12 warps: 3 per SM sub-partition, 16384 / 96 -> 168 registers each at launch.
+__global__ void __launch_bounds__(384, 1)
+    fa_fwd_bf16_2tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const Fwd2Params p) {
+  using C = Fwd2Cfg<HD>;
+  constexpr int ST = C::STAGES;
+  constexpr int KCH = HD / 64;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_q, bar_kfull[ST], bar_kempty[ST], bar_vfull[ST], bar_vempty[ST];
+  __shared__ uint64_t bar_sfull[2], bar_pfull[2], bar_odone[2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sQ = base;  // tile t at sQ + t * Q_TILE_BYTES
+  const uint32_t sK = sQ + 2 * C::Q_TILE_BYTES;
+  const uint32_t sV = sK + ST * C::KV_BYTES;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work item: groups of HEAD_GROUP heads; inside a group the heaviest
+  // (last) tile pairs of every head start first.
+  const int bid = blockIdx.x;
+  const int per_group = C::HEAD_GROUP * p.num_pairs;
+  const int g = bid / per_group;
+  const int heads_in_group = min(C::HEAD_GROUP, p.BH - g * C::HEAD_GROUP);
+  const int r = bid - g * per_group;
+  const int pair = p.num_pairs - 1 - r / heads_in_group;
+  const int bh = g * C::HEAD_GROUP + r % heads_in_group;
+  const int b = bh / p.Hq;
+  const int hq = bh - b * p.Hq;
+  const int bh_kv = b * p.Hkv + hq / (p.Hq / p.Hkv);
+  const int q0 = pair * 2 * C::BM;
+  const int n_kv_total = (p.N + C::BN - 1) / C::BN;
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qs = q0 + t * C::BM;
+    n_t[t] = qs < p.N ? (p.causal ? min(qs / C::BN + 1, n_kv_total) : n_kv_total) : 0;
+  }
+  const int n_max = max(n_t[0], n_t[1]);
+
+  WaitCtl wc{&abort_flag, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar_q), 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(smem_u32(&bar_kfull[s]), 1);
+      mbar_init(smem_u32(&bar_kempty[s]), 1);
+      mbar_init(smem_u32(&bar_vfull[s]), 1);
+      mbar_init(smem_u32(&bar_vempty[s]), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(&bar_sfull[t]), 1);
+      mbar_init(smem_u32(&bar_pfull[t]), 128);
+      mbar_init(smem_u32(&bar_odone[t]), 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
+  }
+  if (warp >= 10) {
+    // idle warps of the third warpgroup
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      const int live_tiles = n_t[1] > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(smem_u32(&bar_q), live_tiles * C::Q_TILE_BYTES);
+      for (int t = 0; t < live_tiles; ++t)
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * (C::BM * 128), &tm_q, smem_u32(&bar_q), c * 64,
+                      q0 + t * C::BM, bh);
+      for (int j = 0; j < n_max; ++j) {
+        const int s = j % ST;
+        const uint32_t ph = (j / ST) & 1;
+        if (!mbar_wait(smem_u32(&bar_kempty[s]), ph ^ 1, wc)) break;
+        mbar_arrive_expect_tx(smem_u32(&bar_kfull[s]), C::KV_BYTES);
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(sK + s * C::KV_BYTES + c * (C::BN * 128), &tm_k, smem_u32(&bar_kfull[s]), c * 64,
+                      j * C::BN, bh_kv);
+        if (!mbar_wait(smem_u32(&bar_vempty[s]), ph ^ 1, wc)) break;
+        mbar_arrive_expect_tx(smem_u32(&bar_vfull[s]), C::KV_BYTES);
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(sV + s * C::KV_BYTES + c * (C::BN * 128), &tm_v, smem_u32(&bar_vfull[s]), c * 64,
+                      j * C::BN, bh_kv);
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, HD, false, true);
+      auto issue_s = [&](int t, int j) {
+        const uint32_t kb = sK + (j % ST) * C::KV_BYTES;
+        const uint32_t qb = sQ + t * C::Q_TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_bf16_ss(tmem + t * 128, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk,
+                      kk > 0);
+        }
+        mma_commit(smem_u32(&bar_sfull[t]));
+      };
+      bool ok = mbar_wait(smem_u32(&bar_q), 0, wc) && mbar_wait(smem_u32(&bar_kfull[0]), 0, wc);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t] > 0) issue_s(t, 0);
+        mma_commit(smem_u32(&bar_kempty[0]));
+      }
+      for (int j = 0; ok && j < n_max; ++j) {
+        const int s = j % ST;
+        bool v_ready = false, k_next_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= n_t[t]) continue;
+          if (!mbar_wait(smem_u32(&bar_pfull[t]), j & 1, wc)) { ok = false; break; }
+          if (!v_ready) {
+            if (!mbar_wait(smem_u32(&bar_vfull[s]), (j / ST) & 1, wc)) { ok = false; break; }
+            v_ready = true;
+          }
+          tc_fence_after();
+          const uint32_t vb = sV + s * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk)
+            mma_bf16_ts(tmem + C::TMEM_O + t * HD, tmem + t * 128 + kk * 8,
+                        sdesc_sw128(vb + kk * 2048, C::BN * 128, 1024), idesc_pv, (j > 0 || kk > 0));
+          mma_commit(smem_u32(&bar_odone[t]));
+          if (j + 1 < n_t[t]) {
+            if (!k_next_ready) {
+              if (!mbar_wait(smem_u32(&bar_kfull[(j + 1) % ST]), ((j + 1) / ST) & 1, wc)) { ok = false; break; }
+              k_next_ready = true;
+              tc_fence_after();
+            }
+            issue_s(t, j + 1);
+          }
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&bar_vempty[s]));
+        if (k_next_ready) mma_commit(smem_u32(&bar_kempty[(j + 1) % ST]));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
+    const int t = warp >> 2;                      // query tile of this warpgroup
+    const int row = q0 + t * C::BM + (threadIdx.x & 127);
+    const uint32_t lane_base = ((warp & 3) * 32u) << 16;
+    const uint32_t s_addr = tmem + lane_base + t * 128;
+    const uint32_t o_addr = tmem + lane_base + C::TMEM_O + t * HD;
+    const int n = n_t[t];
+    const uint64_t c2 = pack2(p.scale_log2, p.scale_log2);
+    float m_ref = -INFINITY;
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      if (!warp_wait(smem_u32(&bar_sfull[t]), j & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld128(s_addr, sr);
+      const int key0 = j * C::BN;
+      if ((p.causal && key0 + C::BN > q0 + t * C::BM) || key0 + C::BN > p.N) {
+        const int lim = min(p.causal ? row + 1 : p.N, p.N) - key0;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
+      }
+      // row max: eight independent three-input chains, then a short tree
+      float mk[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mk[k] = __uint_as_float(sr[k]);
+#pragma unroll
+      for (int c = 8; c < 128; c += 16) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mk[k] = max3f(mk[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+      }
+      const float mx = max3f(max3f(mk[0], mk[1], mk[2]), max3f(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7])) *
+                       p.scale_log2;
+      // Raise the reference maximum only when this tile's maximum exceeds it
+      // by more than the threshold (decided per warp); the running output is
+      // rescaled below, after P is stored, while the score row is dead.
+      bool rescale = false;
+      float alpha = 1.f;
+      if (j == 0) {
+        m_ref = mx;
+      } else if (__any_sync(0xffffffffu, mx > m_ref + C::RESCALE_THRESHOLD)) {
+        const float m_new = fmaxf(m_ref, mx);
+        alpha = ex2_approx(m_ref - m_new);
+        m_ref = m_new;
+        rescale = true;
+      }
+      // p = 2^(s * scale * log2 e - m), packed to bf16 over the S columns
+      const uint64_t negm2 = pack2(-m_ref, -m_ref);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        float x0, x1;
+        unpack2(ffma2(pack2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), c2, negm2), x0, x1);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        acc[c & 3] = fadd2(acc[c & 3], pack2(p0, p1));
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      float s0, s1;
+      unpack2(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), s0, s1);
+      l = l * alpha + (s0 + s1);
+      {
+        uint32_t h0[32], h1[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          h0[i] = pk[i];
+          h1[i] = pk[32 + i];
+        }
+        tmem_st32(s_addr, h0);
+        tmem_st32(s_addr + 32, h1);
+      }
+      if (rescale) {
+        // o was last written by P_{j-1} V_{j-1}: wait for it, then scale by alpha
+        if (!warp_wait(smem_u32(&bar_odone[t]), (j - 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t a2 = pack2(alpha, alpha);
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(o_addr + c * 32, orr);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float lo, hi;
+            unpack2(fmul2(pack2(__uint_as_float(orr[2 * i]), __uint_as_float(orr[2 * i + 1])), a2), lo, hi);
+            orr[2 * i] = __float_as_uint(lo);
+            orr[2 * i + 1] = __float_as_uint(hi);
+          }
+          tmem_st32(o_addr + c * 32, orr);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_pfull[t]));
+    }
+    if (n > 0 && ok && warp_wait(smem_u32(&bar_odone[t]), (n - 1) & 1, wc)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool live = row < p.N;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (live ? row : 0)) * HD;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t orr[32];
+        tmem_ld32(o_addr + c * 32, orr);
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          wp[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = w[i];
+        }
+      }
+      if (live) p.lse[static_cast<size_t>(bh) * p.N + row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa
