@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libfa_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 SOURCES = ["fa_api.cu"]
-HEADERS = ["sm100_ptx.cuh", "fwd_sm100.cuh", "fwd2_sm100.cuh", "fwd_f32.cuh", "bwd_sm100.cuh"]
+HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))
 
 
 def _nvcc() -> str:

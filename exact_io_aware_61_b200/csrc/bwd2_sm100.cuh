@@ -1,0 +1,519 @@
+// bwd2_sm100.cuh -- pipelined recompute backward (bf16, head dimension 64 or
+// 128) for sm_100a.
+//
+// Same arithmetic as the single-warpgroup kernel in bwd_sm100.cuh (rebuild
+// P from the stored LSE, then dV = P^T dO, dS = P * (dP - D), dK = scale
+// dS^T Q, dQ = scale dS K), with the per-step work spread over three
+// warpgroups so that it runs while the tensor core works on other GEMMs:
+//   warps 0-3   "P"  : P^T = exp2(S^T * scale * log2 e - LSE2) -> TMEM (bf16)
+//   warps 4-7   "dS" : dS^T = P^T (dP^T - D) scale -> shared memory (bf16)
+//   warps 8-11  "dQ" : dQ tile TMEM -> registers -> red.global.add.v4.f32
+//   warp 12          : TMA producer (K, V once; Q, LSE2, D double-buffered; dO)
+//   warp 13          : TMEM allocator and MMA issuer
+// MMA order per step t (query tile):
+//   dP^T(t) [after dQ(t-1) left TMEM], dV += P^T dO, dK += dS^T Q,
+//   dQ(t) [into the dP^T columns], then S^T(t+1) at once, so the P warpgroup
+//   can start on step t+1 while the dQ warpgroup drains dQ(t).
+// TMEM: S^T / P^T at 0, dP^T / dQ at 128, dV at 256, dK at 256 + d.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+template <int HD>
+struct Bwd2Cfg {
+  static constexpr int TILE = 128 * HD * 2;  // one 128-row bf16 tile
+  static constexpr int QST = 2;              // stages of (Q, LSE2, D)
+  static constexpr int DOST = HD == 64 ? 2 : 1;
+  static constexpr int QSTAGE_BYTES = TILE + 1024;
+  static constexpr int DS_BYTES = 128 * 128 * 2;
+  // d = 128: 32 query rows of dQ (f32) are staged here for a bulk reduce-add
+  static constexpr int DQ_STAGE_BYTES = HD == 128 ? 32 * 128 * 4 : 0;
+  static constexpr int SMEM_BYTES =
+      1024 + 2 * TILE + QST * QSTAGE_BYTES + DOST * TILE + DS_BYTES + DQ_STAGE_BYTES;
+  static constexpr int THREADS = 448;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S = 0;
+  static constexpr uint32_t T_DP = 128;
+  static constexpr uint32_t T_DV = 256;
+  static constexpr uint32_t T_DK = 256 + HD;
+  // d = 128: the dQ tile is formed transposed (M = d = 128 lanes); d = 64
+  // keeps M = queries, since an M = 64 accumulator has another TMEM layout.
+  static constexpr bool DQ_TRANSPOSED = HD == 128;
+};
+
+struct Bwd2Params {
+  const float* ws_delta;
+  const float* ws_lse2;
+  float* dq_acc;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int N, Npad, Hq, Hkv, num_tiles;
+  float scale_log2;
+  float scale;
+  int causal;
+  unsigned long long timeout_ns;
+};
+
+FA_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+FA_DEV void red_add_v4(float* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+FA_DEV void red_add_f32(float* p, uint32_t a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "r"(a) : "memory");
+}
+
+// TMEM -> registers without waiting; pair with tmem_wait_ld32 on the same
+// registers before using them.
+FA_DEV void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Orders later uses of `r` after the preceding (volatile) wait.
+FA_DEV void tmem_tie32(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+FA_DEV void tmem_ld16_async(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+FA_DEV void tmem_tie16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
+}
+
+// Wait for every outstanding TMEM load of this thread; the registers are
+// tied to the wait so no use of them can move above it.
+FA_DEV void tmem_wait_ld32(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+// 14 warps leave 4 on some SM sub-partitions: 16384 / 128 -> 128 registers.
+template <int HD>
+__global__ void __launch_bounds__(512, 1)
+    fa_bwd2_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const Bwd2Params p) {
+  using C = Bwd2Cfg<HD>;
+  constexpr int QST = C::QST, DOST = C::DOST;
+  constexpr int KCH = HD / 64;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_kv, bar_qfull[QST], bar_qempty[QST], bar_dofull[DOST], bar_doempty[DOST];
+  __shared__ uint64_t bar_sfull, bar_pfull, bar_dpfull, bar_dsfull, bar_dqfull, bar_dqfree, bar_final, bar_dqwg;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* const gbase = smem_raw + (base - smem_u32(smem_raw));
+  const uint32_t sK = base;
+  const uint32_t sV = sK + C::TILE;
+  const uint32_t sQ = sV + C::TILE;                    // stage s: Q at +s*QSTAGE, LSE2/D after Q
+  const uint32_t sDO = sQ + QST * C::QSTAGE_BYTES;
+  const uint32_t sDS = sDO + DOST * C::TILE;
+  const uint32_t sDQ = sDS + C::DS_BYTES;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int bhkv = static_cast<int>(blockIdx.x) / p.num_tiles;
+  const int kt = static_cast<int>(blockIdx.x) - bhkv * p.num_tiles;  // tile 0 has the most work when causal
+  const int k0 = kt * 128;
+  const int b = bhkv / p.Hkv;
+  const int hkv = bhkv - b * p.Hkv;
+  const int group = p.Hq / p.Hkv;
+  const int i_begin = p.causal ? kt : 0;
+  const int per_head = p.num_tiles - i_begin;
+  const int steps = group * per_head;
+
+  WaitCtl wc{&abort_flag, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar_kv), 1);
+    for (int s = 0; s < QST; ++s) {
+      mbar_init(smem_u32(&bar_qfull[s]), 1);
+      mbar_init(smem_u32(&bar_qempty[s]), 1);
+    }
+    for (int s = 0; s < DOST; ++s) {
+      mbar_init(smem_u32(&bar_dofull[s]), 1);
+      mbar_init(smem_u32(&bar_doempty[s]), 1);
+    }
+    mbar_init(smem_u32(&bar_sfull), 1);
+    mbar_init(smem_u32(&bar_pfull), 256);
+    mbar_init(smem_u32(&bar_dpfull), 1);
+    mbar_init(smem_u32(&bar_dsfull), 256);
+    mbar_init(smem_u32(&bar_dqfull), 1);
+    mbar_init(smem_u32(&bar_dqfree), 128);
+    mbar_init(smem_u32(&bar_final), 1);
+    mbar_init(smem_u32(&bar_dqwg), 128);
+    fence_mbar_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(smem_u32(&tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  auto step_tile = [&](int t, int& bhq, int& q0) {
+    const int hh = t / per_head;
+    q0 = (i_begin + (t - hh * per_head)) * 128;
+    bhq = b * p.Hq + hkv * group + hh;
+  };
+
+  if (warp == 12) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_do);
+      mbar_arrive_expect_tx(smem_u32(&bar_kv), 2 * C::TILE);
+      for (int c = 0; c < KCH; ++c) {
+        tma_load_3d(sK + c * 16384, &tm_k, smem_u32(&bar_kv), c * 64, k0, bhkv);
+        tma_load_3d(sV + c * 16384, &tm_v, smem_u32(&bar_kv), c * 64, k0, bhkv);
+      }
+      for (int t = 0; t < steps; ++t) {
+        int bhq, q0;
+        step_tile(t, bhq, q0);
+        const int sq = t % QST, sd = t % DOST;
+        if (!mbar_wait(smem_u32(&bar_qempty[sq]), ((t / QST) & 1) ^ 1, wc)) break;
+        const uint32_t qst = sQ + sq * C::QSTAGE_BYTES;
+        const uint32_t qb = smem_u32(&bar_qfull[sq]);
+        mbar_arrive_expect_tx(qb, C::QSTAGE_BYTES);
+        for (int c = 0; c < KCH; ++c) tma_load_3d(qst + c * 16384, &tm_q, qb, c * 64, q0, bhq);
+        const size_t roff = static_cast<size_t>(bhq) * p.Npad + q0;
+        bulk_load(qst + C::TILE, p.ws_lse2 + roff, 512, qb);
+        bulk_load(qst + C::TILE + 512, p.ws_delta + roff, 512, qb);
+        if (!mbar_wait(smem_u32(&bar_doempty[sd]), ((t / DOST) & 1) ^ 1, wc)) break;
+        const uint32_t db = smem_u32(&bar_dofull[sd]);
+        mbar_arrive_expect_tx(db, C::TILE);
+        for (int c = 0; c < KCH; ++c) tma_load_3d(sDO + sd * C::TILE + c * 16384, &tm_do, db, c * 64, q0, bhq);
+      }
+    }
+  } else if (warp == 13) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t id_kmn = idesc_bf16_f32(128, HD, false, true);   // dV, dK
+      constexpr uint32_t id_mnmn = C::DQ_TRANSPOSED ? idesc_bf16_f32(128, 128, true, true)   // dQ^T
+                                                    : idesc_bf16_f32(128, HD, true, true);   // dQ
+      auto issue_s = [&](int t) {
+        const uint32_t qst = sQ + (t % QST) * C::QSTAGE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + C::T_S, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(qst + off, 16, 1024), id_kk,
+                      kk > 0);
+        }
+        mma_commit(smem_u32(&bar_sfull));
+      };
+      bool ok = mbar_wait(smem_u32(&bar_kv), 0, wc) && mbar_wait(smem_u32(&bar_qfull[0]), 0, wc);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int t = 0; ok && t < steps; ++t) {
+        const int sq = t % QST, sd = t % DOST;
+        const uint32_t qst = sQ + sq * C::QSTAGE_BYTES;
+        const uint32_t dob = sDO + sd * C::TILE;
+        if (t > 0 && !mbar_wait(smem_u32(&bar_dqfree), (t - 1) & 1, wc)) break;
+        if (!mbar_wait(smem_u32(&bar_dofull[sd]), (t / DOST) & 1, wc)) break;
+        tc_fence_after();
+        // dP^T = V dO^T
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + C::T_DP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(dob + off, 16, 1024), id_kk,
+                      kk > 0);
+        }
+        mma_commit(smem_u32(&bar_dpfull));
+        // dV += P^T dO
+        if (!mbar_wait(smem_u32(&bar_pfull), t & 1, wc)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + C::T_DV, tmem + C::T_S + (kk >> 2) * 64 + (kk & 3) * 8,
+                      sdesc_sw128(dob + kk * 2048, 16384, 1024), id_kmn,
+                      (t > 0 || kk > 0));
+        mma_commit(smem_u32(&bar_doempty[sd]));
+        // dK += dS^T Q ; dQ = dS K
+        if (!mbar_wait(smem_u32(&bar_dsfull), t & 1, wc)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + C::T_DK, sdesc_sw128(sDS + off, 16, 1024), sdesc_sw128(qst + kk * 2048, 16384, 1024),
+                      id_kmn, (t > 0 || kk > 0));
+        }
+        if constexpr (C::DQ_TRANSPOSED) {
+          // dQ^T = K^T dS^T (M = d, N = queries): TMEM lane = head-dim index,
+          // so a warp's reduction of one query row is one 128-byte line.
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ss(tmem + C::T_DP, sdesc_sw128(sK + kk * 2048, 16384, 1024),
+                        sdesc_sw128(sDS + kk * 2048, 16384, 1024), id_mnmn, kk > 0);
+        } else {
+          // dQ = dS K (M = queries, N = d)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ss(tmem + C::T_DP, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
+                        sdesc_sw128(sK + kk * 2048, 16384, 1024), id_mnmn, kk > 0);
+        }
+        mma_commit(smem_u32(&bar_qempty[sq]));
+        mma_commit(smem_u32(&bar_dqfull));
+        if (t + 1 < steps) {
+          if (!mbar_wait(smem_u32(&bar_qfull[(t + 1) % QST]), ((t + 1) / QST) & 1, wc)) break;
+          tc_fence_after();
+          issue_s(t + 1);
+        }
+      }
+      mma_commit(smem_u32(&bar_final));
+    }
+  } else if (warp < 8) {
+    // ---------------------------------------------------- compute warpgroups
+    // Warpgroup `half` owns query columns [64 half, 64 half + 64) of every
+    // step: it turns its S^T columns into P^T (bf16, written over its own
+    // S^T columns 64 half .. 64 half + 31) and later its dP^T columns into
+    // dS^T (bf16, shared-memory block `half`). Both warpgroups cover all 128
+    // key rows (TMEM lane = key).
+    const int half = warp >> 2;
+    const int tid = threadIdx.x & 127;  // key row k0 + tid
+    const int cb = half * 64;           // first query column of this warpgroup
+    const uint32_t lane_base = ((warp & 3) * 32u) << 16;
+    const int key = k0 + tid;
+    const bool key_live = key < p.N;
+    uint8_t* ds_row = gbase + (sDS - base) + half * 16384 + tid * 128;
+    bool ok = true;
+    for (int t = 0; t < steps; ++t) {
+      int bhq, q0;
+      step_tile(t, bhq, q0);
+      const int sq = t % QST;
+      const float* lse2 = reinterpret_cast<const float*>(gbase + (sQ - base) + sq * C::QSTAGE_BYTES + C::TILE);
+      const float4* l4 = reinterpret_cast<const float4*>(lse2 + cb);
+      const float4* d4 = reinterpret_cast<const float4*>(lse2 + 128 + cb);
+      if (!warp_wait(smem_u32(&bar_qfull[sq]), (t / QST) & 1, wc)) { ok = false; break; }
+      if (!warp_wait(smem_u32(&bar_sfull), t & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      // ---- P^T = exp2(S^T * scale * log2 e - LSE2), masked
+      const bool diag = p.causal && (q0 == k0);
+      {
+        uint32_t rr[2][32];
+        tmem_ld32_async(tmem + lane_base + C::T_S + cb, rr[0]);
+        tmem_ld32_async(tmem + lane_base + C::T_S + cb + 32, rr[1]);
+        tmem_wait_ld32(rr[0]);
+        tmem_tie32(rr[1]);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const float4 L = l4[u * 8 + x];
+            const int qa = cb + u * 32 + 4 * x;  // query column of element 0
+            float pv[4];
+            pv[0] = ex2_approx(fmaf(__uint_as_float(rr[u][4 * x]), p.scale_log2, -L.x));
+            pv[1] = ex2_approx(fmaf(__uint_as_float(rr[u][4 * x + 1]), p.scale_log2, -L.y));
+            pv[2] = ex2_approx(fmaf(__uint_as_float(rr[u][4 * x + 2]), p.scale_log2, -L.z));
+            pv[3] = ex2_approx(fmaf(__uint_as_float(rr[u][4 * x + 3]), p.scale_log2, -L.w));
+            if (diag) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (q0 + qa + e < key) pv[e] = 0.f;
+            }
+            pk[2 * x] = key_live ? pack_bf16x2(pv[0], pv[1]) : 0u;
+            pk[2 * x + 1] = key_live ? pack_bf16x2(pv[2], pv[3]) : 0u;
+          }
+          tmem_st16(tmem + lane_base + C::T_S + cb + u * 16, pk);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_pfull));
+      // ---- dS^T = P^T (dP^T - D) * scale -> shared memory
+      if (t > 0 && !warp_wait(smem_u32(&bar_dqfull), (t - 1) & 1, wc)) { ok = false; break; }  // dS(t-1) consumed
+      if (!warp_wait(smem_u32(&bar_dpfull), t & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        uint32_t r[32], pr[16];
+        tmem_ld32_async(tmem + lane_base + C::T_DP + cb + u * 32, r);
+        tmem_ld16_async(tmem + lane_base + C::T_S + cb + u * 16, pr);
+        tmem_wait_ld32(r);
+        tmem_tie16(pr);
+        uint32_t w[16];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const float4 Dv = d4[u * 8 + x];
+          const float e0 = bf16_lo(pr[2 * x]) * (__uint_as_float(r[4 * x]) - Dv.x) * p.scale;
+          const float e1 = bf16_hi(pr[2 * x]) * (__uint_as_float(r[4 * x + 1]) - Dv.y) * p.scale;
+          const float e2 = bf16_lo(pr[2 * x + 1]) * (__uint_as_float(r[4 * x + 2]) - Dv.z) * p.scale;
+          const float e3 = bf16_hi(pr[2 * x + 1]) * (__uint_as_float(r[4 * x + 3]) - Dv.w) * p.scale;
+          w[2 * x] = pack_bf16x2(e0, e1);
+          w[2 * x + 1] = pack_bf16x2(e2, e3);
+        }
+        // 32 queries = 64 bytes = four 16-byte chunks: chunk u*4 + v, swizzled by row
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int chunk = (u * 4 + v) ^ (tid & 7);
+          *reinterpret_cast<uint4*>(ds_row + chunk * 16) = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_dsfull));
+    }
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (dS carries the scale)
+    if (ok && warp_wait(smem_u32(&bar_final), 0, wc)) {
+      tc_fence_after();
+      __nv_bfloat16* out = (half == 0 ? p.dv : p.dk) + (static_cast<size_t>(bhkv) * p.N + (key_live ? key : 0)) * HD;
+      const uint32_t col = half == 0 ? C::T_DV : C::T_DK;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + col + c * 32, r);
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int x = 0; x < 16; ++x) wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]), __uint_as_float(r[2 * x + 1]));
+        if (key_live) {
+#pragma unroll
+          for (int x = 0; x < 4; ++x) reinterpret_cast<uint4*>(out + c * 32)[x] = w[x];
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------- dQ warpgroup
+    const int tid = threadIdx.x - 256;  // d index (transposed dQ) or query row q0 + tid
+    const uint32_t lane_base = ((warp & 3) * 32u) << 16;
+    uint32_t wg_phase = 0;
+    auto wg_sync = [&]() -> bool {  // bounded barrier over the 128 dQ threads
+      mbar_arrive(smem_u32(&bar_dqwg));
+      const bool r = warp_wait(smem_u32(&bar_dqwg), wg_phase, wc);
+      wg_phase ^= 1u;
+      return r;
+    };
+    bool ok = true;
+    for (int t = 0; t < steps && ok; ++t) {
+      int bhq, q0;
+      step_tile(t, bhq, q0);
+      if (!warp_wait(smem_u32(&bar_dqfull), t & 1, wc)) break;
+      tc_fence_after();
+      if constexpr (C::DQ_TRANSPOSED) {
+        // Thread tid holds dQ[q0 + j][tid] in TMEM column j. The tile leaves
+        // TMEM in two halves of 64 query columns; once both halves are in
+        // registers the columns are released to the next dP^T. Each 32-row
+        // chunk is then written row-major to shared memory (a warp writes
+        // 128 contiguous bytes per row) and added to the accumulator with one
+        // asynchronous bulk reduce-add.
+        float* stage = reinterpret_cast<float*>(gbase + (sDQ - base));
+        float* rows = p.dq_acc + static_cast<size_t>(bhq) * p.N * HD;
+#pragma unroll
+        for (int h = 0; h < 2 && ok; ++h) {
+          uint32_t rr[2][32];
+          tmem_ld32_async(tmem + lane_base + C::T_DP + h * 64, rr[0]);
+          tmem_ld32_async(tmem + lane_base + C::T_DP + h * 64 + 32, rr[1]);
+          tmem_wait_ld32(rr[0]);
+          tmem_tie32(rr[1]);
+          if (h == 1) {
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bar_dqfree));
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int r0 = q0 + (2 * h + u) * 32;
+            const int nrows = min(32, p.N - r0);
+            if (tid == 0) bulk_wait_group_read<0>();  // staging buffer read by the last reduce
+            if (!wg_sync()) { ok = false; break; }
+            if (nrows > 0) {
+#pragma unroll
+              for (int x = 0; x < 32; ++x) stage[x * 128 + tid] = __uint_as_float(rr[u][x]);
+            }
+            fence_proxy_async_smem();
+            if (!wg_sync()) { ok = false; break; }
+            if (tid == 0 && nrows > 0) {
+              bulk_reduce_add_f32(rows + static_cast<size_t>(r0) * HD, sDQ, static_cast<uint32_t>(nrows) * HD * 4);
+              bulk_commit_group();
+            }
+          }
+        }
+        continue;
+      } else {
+        const int row = q0 + tid;
+        const bool live = row < p.N;
+        float* dst = p.dq_acc + (static_cast<size_t>(bhq) * p.N + (live ? row : 0)) * HD;
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + C::T_DP + c * 32, r);
+          if (live) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              red_add_v4(dst + c * 32 + 4 * u, r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bar_dqfree));
+      }
+    }
+    if (tid == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

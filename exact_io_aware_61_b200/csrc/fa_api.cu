@@ -21,6 +21,7 @@
 #include "fwd2_sm100.cuh"
 #include "fwd_f32.cuh"
 #include "bwd_sm100.cuh"
+#include "bwd2_sm100.cuh"
 
 namespace {
 
@@ -84,8 +85,8 @@ int prepare_kernels(int dev) {
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<64>), fa::fwd_f32_smem_bytes<64>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<128>), fa::fwd_f32_smem_bytes<128>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<256>), fa::fwd_f32_smem_bytes<256>());
-  set(reinterpret_cast<const void*>(&fa::fa_bwd_main_kernel<64>), fa::BwdCfg<64>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_bwd_main_kernel<128>), fa::BwdCfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64>), fa::Bwd2Cfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128>), fa::Bwd2Cfg<128>::SMEM_BYTES);
   if (e != cudaSuccess) return FA_ERR_CUDA;
   done[dev] = true;
   return FA_OK;
@@ -283,20 +284,20 @@ int launch_bwd_prep(const void* o, const float* lse, const void* dO, void* ws, i
 template <int HD>
 int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* ws,
                     int B, int Hq, int Hkv, int N, float scale, int causal, cudaStream_t stream) {
-  using C = fa::BwdCfg<HD>;
+  using C = fa::Bwd2Cfg<HD>;
   const BwdWorkspace w = carve(ws, B, Hq, N);
   const size_t npad = padded_rows(N);
   const uint64_t rows_q = static_cast<uint64_t>(B) * Hq, rows_kv = static_cast<uint64_t>(B) * Hkv;
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo;
   int rc = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
   if (rc == FA_OK) rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
   if (rc == FA_OK) rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
   if (rc == FA_OK) rc = make_map(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
-  if (rc == FA_OK) rc = make_map(&mdq, w.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, N, rows_q, 32, 128);
   if (rc != FA_OK) return rc;
-  fa::BwdParams p;
+  fa::Bwd2Params p;
   p.ws_delta = w.delta;
   p.ws_lse2 = w.lse2;
+  p.dq_acc = w.dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.N = N;
@@ -310,9 +311,9 @@ int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO,
   p.timeout_ns = timeout_now();
   const long long blocks = static_cast<long long>(p.num_tiles) * B * Hkv;
   if (blocks > INT32_MAX) return FA_ERR_INVALID;
-  fa::fa_bwd_main_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
-                                                                                                    mdq, p);
-  return launch_status();
+  fa::fa_bwd2_main_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
+                                                                                                     p);
+  return launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>));
 }
 
 int launch_bwd_dq(void* dq, void* ws, int B, int Hq, int N, int d, cudaStream_t stream) {

@@ -49,14 +49,19 @@ FA_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
                : "memory");
 }
 
+// One bounded probe of the phase; the waiting thread may be suspended by the
+// hardware for up to kSuspendHintNs (it resumes as soon as the phase
+// completes), so waiting warps do not take issue slots from working ones.
+constexpr uint32_t kSuspendHintNs = 20000;
+
 FA_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.b32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "n"(kSuspendHintNs)
       : "memory");
   return done != 0;
 }
@@ -124,6 +129,14 @@ FA_DEV void tma_reduce_add_3d(const void* tmap, uint32_t src, int x, int y, int 
       " [%0, {%1, %2, %3}], [%4];" ::"l"(tmap),
       "r"(x), "r"(y), "r"(z), "r"(src)
       : "memory");
+}
+
+// Contiguous bulk reduce-add of f32 values shared -> global (both addresses
+// 16-byte aligned, size % 16 == 0).
+FA_DEV void bulk_reduce_add_f32(float* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc),
+               "r"(bytes)
+               : "memory");
 }
 
 FA_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
