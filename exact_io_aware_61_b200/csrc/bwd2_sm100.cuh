@@ -34,7 +34,15 @@ struct Bwd2Cfg {
   static constexpr int DQ_STAGE_BYTES = HD == 128 ? 32 * 128 * 4 : 0;
   static constexpr int SMEM_BYTES =
       1024 + 2 * TILE + QST * QSTAGE_BYTES + DOST * TILE + DS_BYTES + DQ_STAGE_BYTES;
-  static constexpr int THREADS = 448;
+  static constexpr int THREADS = 512;
+  // Launch with 128 registers per thread (16 warps, 4 per SM sub-partition),
+  // then redistribute per warpgroup: 128 x (120 + 120 + 168 + 104) = 512 x 128.
+  static constexpr int LAUNCH_REGS = 128;
+  static constexpr int COMPUTE_REGS = 120;
+  static constexpr int DRAIN_REGS = 168;
+  static constexpr int OTHER_REGS = 104;
+  static_assert(128 * (2 * COMPUTE_REGS + DRAIN_REGS + OTHER_REGS) <= THREADS * LAUNCH_REGS,
+                "register split exceeds the launch allocation");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0;
   static constexpr uint32_t T_DP = 128;
@@ -137,7 +145,7 @@ FA_DEV void tmem_wait_ld32(uint32_t (&r)[32]) {
                : "memory");
 }
 
-// 14 warps leave 4 on some SM sub-partitions: 16384 / 128 -> 128 registers.
+// 16 warps, 4 per SM sub-partition: 16384 / 128 -> 128 registers at launch.
 template <int HD>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd2_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -213,7 +221,9 @@ __global__ void __launch_bounds__(512, 1)
     bhq = b * p.Hq + hkv * group + hh;
   };
 
-  if (warp == 12) {
+  if (warp >= 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
+    if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -320,7 +330,9 @@ __global__ void __launch_bounds__(512, 1)
       }
       mma_commit(smem_u32(&bar_final));
     }
+    }  // warps 14, 15: idle
   } else if (warp < 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::COMPUTE_REGS));
     // ---------------------------------------------------- compute warpgroups
     // Warpgroup `half` owns query columns [64 half, 64 half + 64) of every
     // step: it turns its S^T columns into P^T (bf16, written over its own
@@ -349,12 +361,9 @@ __global__ void __launch_bounds__(512, 1)
       const bool diag = p.causal && (q0 == k0);
       {
         uint32_t rr[2][32];
-        tmem_ld32_async(tmem + lane_base + C::T_S + cb, rr[0]);
-        tmem_ld32_async(tmem + lane_base + C::T_S + cb + 32, rr[1]);
-        tmem_wait_ld32(rr[0]);
-        tmem_tie32(rr[1]);
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
+          tmem_ld32(tmem + lane_base + C::T_S + cb + 32 * u, rr[u]);
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
@@ -432,6 +441,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::DRAIN_REGS));
     // ------------------------------------------------------- dQ warpgroup
     const int tid = threadIdx.x - 256;  // d index (transposed dQ) or query row q0 + tid
     const uint32_t lane_base = ((warp & 3) * 32u) << 16;
@@ -457,33 +467,33 @@ __global__ void __launch_bounds__(512, 1)
         // asynchronous bulk reduce-add.
         float* stage = reinterpret_cast<float*>(gbase + (sDQ - base));
         float* rows = p.dq_acc + static_cast<size_t>(bhq) * p.N * HD;
+        uint32_t rr[4][32];
+        tmem_ld32_async(tmem + lane_base + C::T_DP, rr[0]);
+        tmem_ld32_async(tmem + lane_base + C::T_DP + 32, rr[1]);
+        tmem_ld32_async(tmem + lane_base + C::T_DP + 64, rr[2]);
+        tmem_ld32_async(tmem + lane_base + C::T_DP + 96, rr[3]);
+        tmem_wait_ld32(rr[0]);
+        tmem_tie32(rr[1]);
+        tmem_tie32(rr[2]);
+        tmem_tie32(rr[3]);
+        // the whole tile is in registers: release the columns to dP^T(t+1)
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bar_dqfree));
 #pragma unroll
-        for (int h = 0; h < 2 && ok; ++h) {
-          uint32_t rr[2][32];
-          tmem_ld32_async(tmem + lane_base + C::T_DP + h * 64, rr[0]);
-          tmem_ld32_async(tmem + lane_base + C::T_DP + h * 64 + 32, rr[1]);
-          tmem_wait_ld32(rr[0]);
-          tmem_tie32(rr[1]);
-          if (h == 1) {
-            tc_fence_before();
-            mbar_arrive(smem_u32(&bar_dqfree));
+        for (int c = 0; c < 4; ++c) {
+          const int r0 = q0 + c * 32;
+          const int nrows = min(32, p.N - r0);
+          if (tid == 0) bulk_wait_group_read<0>();  // staging buffer read by the last reduce
+          if (!wg_sync()) { ok = false; break; }
+          if (nrows > 0) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) stage[x * 128 + tid] = __uint_as_float(rr[c][x]);
           }
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int r0 = q0 + (2 * h + u) * 32;
-            const int nrows = min(32, p.N - r0);
-            if (tid == 0) bulk_wait_group_read<0>();  // staging buffer read by the last reduce
-            if (!wg_sync()) { ok = false; break; }
-            if (nrows > 0) {
-#pragma unroll
-              for (int x = 0; x < 32; ++x) stage[x * 128 + tid] = __uint_as_float(rr[u][x]);
-            }
-            fence_proxy_async_smem();
-            if (!wg_sync()) { ok = false; break; }
-            if (tid == 0 && nrows > 0) {
-              bulk_reduce_add_f32(rows + static_cast<size_t>(r0) * HD, sDQ, static_cast<uint32_t>(nrows) * HD * 4);
-              bulk_commit_group();
-            }
+          fence_proxy_async_smem();
+          if (!wg_sync()) { ok = false; break; }
+          if (tid == 0 && nrows > 0) {
+            bulk_reduce_add_f32(rows + static_cast<size_t>(r0) * HD, sDQ, static_cast<uint32_t>(nrows) * HD * 4);
+            bulk_commit_group();
           }
         }
         continue;

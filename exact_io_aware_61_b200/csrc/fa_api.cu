@@ -311,6 +311,16 @@ int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO,
   p.timeout_ns = timeout_now();
   const long long blocks = static_cast<long long>(p.num_tiles) * B * Hkv;
   if (blocks > INT32_MAX) return FA_ERR_INVALID;
+  // The kernel redistributes registers between warpgroups (setmaxnreg) on
+  // the assumption of exactly LAUNCH_REGS per thread at launch.
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (attr.numRegs != C::LAUNCH_REGS) {
+    if (verbose()) std::fprintf(stderr, "fa: backward built with %d registers, expected %d\n", attr.numRegs,
+                                C::LAUNCH_REGS);
+    return FA_ERR_UNSUPPORTED;
+  }
   fa::fa_bwd2_main_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
                                                                                                      p);
   return launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>));
