@@ -30,8 +30,8 @@ struct Bwd2Cfg {
   static constexpr int DOST = HD == 64 ? 2 : 1;
   static constexpr int QSTAGE_BYTES = TILE + 1024;
   static constexpr int DS_BYTES = 128 * 128 * 2;
-  // d = 128: 32 query rows of dQ (f32) are staged here for a bulk reduce-add
-  static constexpr int DQ_STAGE_BYTES = HD == 128 ? 32 * 128 * 4 : 0;
+  // one 128-row x 32-column f32 box of the dQ tile, staged for a TMA reduce-add
+  static constexpr int DQ_STAGE_BYTES = 128 * 32 * 4;
   static constexpr int SMEM_BYTES =
       1024 + 2 * TILE + QST * QSTAGE_BYTES + DOST * TILE + DS_BYTES + DQ_STAGE_BYTES;
   static constexpr int THREADS = 512;
@@ -48,9 +48,6 @@ struct Bwd2Cfg {
   static constexpr uint32_t T_DP = 128;
   static constexpr uint32_t T_DV = 256;
   static constexpr uint32_t T_DK = 256 + HD;
-  // d = 128: the dQ tile is formed transposed (M = d = 128 lanes); d = 64
-  // keeps M = queries, since an M = 64 accumulator has another TMEM layout.
-  static constexpr bool DQ_TRANSPOSED = HD == 128;
 };
 
 struct Bwd2Params {
@@ -150,14 +147,14 @@ template <int HD>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd2_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                        const Bwd2Params p) {
+                        const __grid_constant__ CUtensorMap tm_dq, const Bwd2Params p) {
   using C = Bwd2Cfg<HD>;
   constexpr int QST = C::QST, DOST = C::DOST;
   constexpr int KCH = HD / 64;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_kv, bar_qfull[QST], bar_qempty[QST], bar_dofull[DOST], bar_doempty[DOST];
-  __shared__ uint64_t bar_sfull, bar_pfull, bar_dpfull, bar_dsfull, bar_dqfull, bar_dqfree, bar_final, bar_dqwg;
+  __shared__ uint64_t bar_sfull, bar_pfull, bar_dpfull, bar_dsfull, bar_dqfull, bar_dqfree, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -203,7 +200,6 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(smem_u32(&bar_dqfull), 1);
     mbar_init(smem_u32(&bar_dqfree), 128);
     mbar_init(smem_u32(&bar_final), 1);
-    mbar_init(smem_u32(&bar_dqwg), 128);
     fence_mbar_init();
   }
   if (warp == 13) {
@@ -256,8 +252,7 @@ __global__ void __launch_bounds__(512, 1)
     if (lane == 0) {
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t id_kmn = idesc_bf16_f32(128, HD, false, true);   // dV, dK
-      constexpr uint32_t id_mnmn = C::DQ_TRANSPOSED ? idesc_bf16_f32(128, 128, true, true)   // dQ^T
-                                                    : idesc_bf16_f32(128, HD, true, true);   // dQ
+      constexpr uint32_t id_mnmn = idesc_bf16_f32(128, HD, true, true);   // dQ
       auto issue_s = [&](int t) {
         const uint32_t qst = sQ + (t % QST) * C::QSTAGE_BYTES;
 #pragma unroll
@@ -306,20 +301,11 @@ __global__ void __launch_bounds__(512, 1)
           mma_bf16_ss(tmem + C::T_DK, sdesc_sw128(sDS + off, 16, 1024), sdesc_sw128(qst + kk * 2048, 16384, 1024),
                       id_kmn, (t > 0 || kk > 0));
         }
-        if constexpr (C::DQ_TRANSPOSED) {
-          // dQ^T = K^T dS^T (M = d, N = queries): TMEM lane = head-dim index,
-          // so a warp's reduction of one query row is one 128-byte line.
+        // dQ = dS K (M = queries, N = d)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ss(tmem + C::T_DP, sdesc_sw128(sK + kk * 2048, 16384, 1024),
-                        sdesc_sw128(sDS + kk * 2048, 16384, 1024), id_mnmn, kk > 0);
-        } else {
-          // dQ = dS K (M = queries, N = d)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ss(tmem + C::T_DP, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
-                        sdesc_sw128(sK + kk * 2048, 16384, 1024), id_mnmn, kk > 0);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(tmem + C::T_DP, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
+                      sdesc_sw128(sK + kk * 2048, 16384, 1024), id_mnmn, kk > 0);
         mma_commit(smem_u32(&bar_qempty[sq]));
         mma_commit(smem_u32(&bar_dqfull));
         if (t + 1 < steps) {
@@ -443,76 +429,52 @@ __global__ void __launch_bounds__(512, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::DRAIN_REGS));
     // ------------------------------------------------------- dQ warpgroup
-    const int tid = threadIdx.x - 256;  // d index (transposed dQ) or query row q0 + tid
+    // Thread tid holds query row q0 + tid of the dQ tile (TMEM lane = row).
+    // The whole tile is loaded into registers and its columns released to
+    // dP^T(t+1) at once; then, 32 head-dim columns at a time, the rows are
+    // written to a 128-byte-swizzled staging box (one 16-byte vector per
+    // store) and added to the f32 accumulator with a TMA tensor reduce-add,
+    // which also drops rows past N.
+    //
+    // The four warps synchronise with a hardware named barrier. Every warp
+    // runs the same number of barriers whatever happens (a bounded wait that
+    // gives up only clears `ok`, which skips work, never barriers), so a
+    // timeout cannot leave a warp waiting at a barrier for ever.
+    const int tid = threadIdx.x - 256;
     const uint32_t lane_base = ((warp & 3) * 32u) << 16;
-    uint32_t wg_phase = 0;
-    auto wg_sync = [&]() -> bool {  // bounded barrier over the 128 dQ threads
-      mbar_arrive(smem_u32(&bar_dqwg));
-      const bool r = warp_wait(smem_u32(&bar_dqwg), wg_phase, wc);
-      wg_phase ^= 1u;
-      return r;
-    };
+    uint8_t* stage_row = gbase + (sDQ - base) + tid * 128;
     bool ok = true;
-    for (int t = 0; t < steps && ok; ++t) {
+    for (int t = 0; t < steps; ++t) {
       int bhq, q0;
       step_tile(t, bhq, q0);
-      if (!warp_wait(smem_u32(&bar_dqfull), t & 1, wc)) break;
-      tc_fence_after();
-      if constexpr (C::DQ_TRANSPOSED) {
-        // Thread tid holds dQ[q0 + j][tid] in TMEM column j. The tile leaves
-        // TMEM in two halves of 64 query columns; once both halves are in
-        // registers the columns are released to the next dP^T. Each 32-row
-        // chunk is then written row-major to shared memory (a warp writes
-        // 128 contiguous bytes per row) and added to the accumulator with one
-        // asynchronous bulk reduce-add.
-        float* stage = reinterpret_cast<float*>(gbase + (sDQ - base));
-        float* rows = p.dq_acc + static_cast<size_t>(bhq) * p.N * HD;
-        uint32_t rr[4][32];
-        tmem_ld32_async(tmem + lane_base + C::T_DP, rr[0]);
-        tmem_ld32_async(tmem + lane_base + C::T_DP + 32, rr[1]);
-        tmem_ld32_async(tmem + lane_base + C::T_DP + 64, rr[2]);
-        tmem_ld32_async(tmem + lane_base + C::T_DP + 96, rr[3]);
+      ok = warp_wait(smem_u32(&bar_dqfull), t & 1, wc) && ok;
+      uint32_t rr[HD / 32][32];
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) tmem_ld32_async(tmem + lane_base + C::T_DP + c * 32, rr[c]);
         tmem_wait_ld32(rr[0]);
-        tmem_tie32(rr[1]);
-        tmem_tie32(rr[2]);
-        tmem_tie32(rr[3]);
-        // the whole tile is in registers: release the columns to dP^T(t+1)
+#pragma unroll
+        for (int c = 1; c < HD / 32; ++c) tmem_tie32(rr[c]);
         tc_fence_before();
-        mbar_arrive(smem_u32(&bar_dqfree));
+        mbar_arrive(smem_u32(&bar_dqfree));  // the tile is in registers
+      }
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int r0 = q0 + c * 32;
-          const int nrows = min(32, p.N - r0);
-          if (tid == 0) bulk_wait_group_read<0>();  // staging buffer read by the last reduce
-          if (!wg_sync()) { ok = false; break; }
-          if (nrows > 0) {
+      for (int c = 0; c < HD / 32; ++c) {
+        if (tid == 0) bulk_wait_group_read<0>();  // the last reduce has read the staging box
+        named_bar_sync(1, 128);
+        if (ok) {
 #pragma unroll
-            for (int x = 0; x < 32; ++x) stage[x * 128 + tid] = __uint_as_float(rr[c][x]);
-          }
-          fence_proxy_async_smem();
-          if (!wg_sync()) { ok = false; break; }
-          if (tid == 0 && nrows > 0) {
-            bulk_reduce_add_f32(rows + static_cast<size_t>(r0) * HD, sDQ, static_cast<uint32_t>(nrows) * HD * 4);
-            bulk_commit_group();
-          }
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(stage_row + ((u ^ (tid & 7)) * 16)) =
+                make_uint4(rr[c][4 * u], rr[c][4 * u + 1], rr[c][4 * u + 2], rr[c][4 * u + 3]);
         }
-        continue;
-      } else {
-        const int row = q0 + tid;
-        const bool live = row < p.N;
-        float* dst = p.dq_acc + (static_cast<size_t>(bhq) * p.N + (live ? row : 0)) * HD;
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + C::T_DP + c * 32, r);
-          if (live) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              red_add_v4(dst + c * 32 + 4 * u, r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
-          }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (tid == 0 && ok) {
+          tma_reduce_add_3d(&tm_dq, sDQ, c * 32, q0, bhq);
+          bulk_commit_group();
         }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&bar_dqfree));
       }
     }
     if (tid == 0) bulk_wait_all();

@@ -288,11 +288,12 @@ int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO,
   const BwdWorkspace w = carve(ws, B, Hq, N);
   const size_t npad = padded_rows(N);
   const uint64_t rows_q = static_cast<uint64_t>(B) * Hq, rows_kv = static_cast<uint64_t>(B) * Hkv;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   int rc = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
   if (rc == FA_OK) rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
   if (rc == FA_OK) rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
   if (rc == FA_OK) rc = make_map(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
+  if (rc == FA_OK) rc = make_map(&mdq, w.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, N, rows_q, 32, 128);
   if (rc != FA_OK) return rc;
   fa::Bwd2Params p;
   p.ws_delta = w.delta;
@@ -322,7 +323,7 @@ int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO,
     return FA_ERR_UNSUPPORTED;
   }
   fa::fa_bwd2_main_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
-                                                                                                     p);
+                                                                                                     mdq, p);
   return launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>));
 }
 
