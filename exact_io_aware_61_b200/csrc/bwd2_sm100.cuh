@@ -1,19 +1,31 @@
 // bwd2_sm100.cuh -- pipelined recompute backward (bf16, head dimension 64 or
 // 128) for sm_100a.
 //
-// Same arithmetic as the single-warpgroup kernel in bwd_sm100.cuh (rebuild
-// P from the stored LSE, then dV = P^T dO, dS = P * (dP - D), dK = scale
-// dS^T Q, dQ = scale dS K), with the per-step work spread over three
-// warpgroups so that it runs while the tensor core works on other GEMMs:
-//   warps 0-3   "P"  : P^T = exp2(S^T * scale * log2 e - LSE2) -> TMEM (bf16)
-//   warps 4-7   "dS" : dS^T = P^T (dP^T - D) scale -> shared memory (bf16)
-//   warps 8-11  "dQ" : dQ tile TMEM -> registers -> red.global.add.v4.f32
-//   warp 12          : TMA producer (K, V once; Q, LSE2, D double-buffered; dO)
-//   warp 13          : TMEM allocator and MMA issuer
+// The forward keeps only O and the per-row log-sum-exp; the backward
+// recomputes every score tile from Q and K and rebuilds the weights from the
+// stored statistics without a second pass (fanfani.net "FlashAttention", "The
+// backward pass, and where the memory saving comes from"; synthetic.wiki
+// "FlashAttention: attention's bottleneck is the wire, not the maths", "The
+// backward pass buys memory with recompute"). The gradient is the textbook
+// derivative of the softmax:
+//   P  = exp(scale S - LSE)         dV = P^T dO
+//   dP = dO V^T                     D  = rowsum(dO * O)   (prep kernel)
+//   dS = P * (dP - D)               dQ = scale dS K,  dK = scale dS^T Q
+//
+// One CTA per (128-key tile, batch, KV head); it loops over the query heads
+// of the group and the query tiles that see its key tile. Roles (16 warps):
+//   warps 0-7   two compute warpgroups; warpgroup h owns query columns
+//               [64h, 64h + 64): P^T = exp2(S^T * scale * log2 e - LSE2) ->
+//               bf16 over its own S^T columns in TMEM, then
+//               dS^T = P^T (dP^T - D) scale -> shared memory (bf16)
+//   warps 8-11  dQ drain: the dQ tile leaves TMEM at once, then is added to
+//               the f32 accumulator with TMA tensor reduce-adds
+//   warp 12     TMA producer (K, V once; Q, LSE2, D double-buffered; dO)
+//   warp 13     TMEM allocator and MMA issuer; warps 14, 15 idle
 // MMA order per step t (query tile):
-//   dP^T(t) [after dQ(t-1) left TMEM], dV += P^T dO, dK += dS^T Q,
-//   dQ(t) [into the dP^T columns], then S^T(t+1) at once, so the P warpgroup
-//   can start on step t+1 while the dQ warpgroup drains dQ(t).
+//   dP^T(t) [once dQ(t-1) left TMEM], dV += P^T dO, dK += dS^T Q,
+//   dQ(t) [into the dP^T columns], then S^T(t+1) at once, so the compute
+//   warpgroups start on step t+1 while the drain empties dQ(t).
 // TMEM: S^T / P^T at 0, dP^T / dQ at 128, dV at 256, dK at 256 + d.
 #pragma once
 
@@ -62,26 +74,6 @@ struct Bwd2Params {
   int causal;
   unsigned long long timeout_ns;
 };
-
-FA_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
-
-FA_DEV void red_add_v4(float* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-
-FA_DEV void red_add_f32(float* p, uint32_t a) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "r"(a) : "memory");
-}
 
 // TMEM -> registers without waiting; pair with tmem_wait_ld32 on the same
 // registers before using them.

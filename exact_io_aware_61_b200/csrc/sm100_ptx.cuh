@@ -22,8 +22,6 @@ FA_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-FA_DEV uint32_t lane_id() { return threadIdx.x & 31; }
-
 FA_DEV uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -129,14 +127,6 @@ FA_DEV void tma_reduce_add_3d(const void* tmap, uint32_t src, int x, int y, int 
       " [%0, {%1, %2, %3}], [%4];" ::"l"(tmap),
       "r"(x), "r"(y), "r"(z), "r"(src)
       : "memory");
-}
-
-// Contiguous bulk reduce-add of f32 values shared -> global (both addresses
-// 16-byte aligned, size % 16 == 0).
-FA_DEV void bulk_reduce_add_f32(float* gdst, uint32_t ssrc, uint32_t bytes) {
-  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc),
-               "r"(bytes)
-               : "memory");
 }
 
 FA_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
