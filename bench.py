@@ -44,7 +44,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Measured DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
 # of the dominant kernel, with the hash of the kernel source it was taken on.
 # Reported only while the source still hashes to the same value.
-TRAFFIC = {}
+TRAFFIC = {
+    # ncu --set full, benchmark shape, profiles/fa_bwd2_main_kernel_d128_causal_b2_h32_n8192.md
+    "bwd_main": {"src": "e18d9838abad2987", "bytes": 809_591_552 + 491_689_984},
+}
 
 
 def fwd_flops(B, Hq, N, d, causal):
@@ -322,6 +325,28 @@ def run_ours(args, rank, world, local):
     value = world * step_flops * args.steps / (max_ms / 1e3) / 1e12
     bwd_ms = per_kernel["bwd_prep"] + per_kernel["bwd_main"] + per_kernel["bwd_dq"]
 
+    # forward alone: its own timed region (no backward kernels in between)
+    fwd_only = None
+    if not args.no_fwd_only:
+        for _ in range(args.warmup):
+            fa.fa_fwd(q, k, v, o, lse, CAUSAL, scale, stream)
+        fsampler = ClockSampler(physical_gpu_index(local))
+        fsampler.start()
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_fwd = max(args.steps, 20)
+        f0.record(stream)
+        for _ in range(n_fwd):
+            fa.fa_fwd(q, k, v, o, lse, CAUSAL, scale, stream)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        fclocks = fsampler.stop()
+        fwd_ms = max_over_ranks(f0.elapsed_time(f1), world, dev) / n_fwd
+        fwd_only = {"launches": n_fwd, "ms": fwd_ms,
+                    "tflops": world * fwd_flops(B, Hq, N, d, CAUSAL) / fwd_ms / 1e9, "clocks": fclocks}
+
     # end to end through the C ABI: pinned host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
@@ -402,7 +427,7 @@ def run_ours(args, rank, world, local):
                         "step": round(100 * value / world / peak_tf, 2),
                         "peak_tflops": peak_tf, "peak_source": f"{peak_src} bf16_tflops (burst)"},
         "kernels": {k: {kk: round(vv, 4) for kk, vv in v.items()} for k, v in kernels.items()},
-        "roofline": {"kernel": "fa_bwd_main_kernel<128>" if dominant == "bwd_main" else "fa_fwd_bf16_kernel<128>",
+        "roofline": {"kernel": f"fa_bwd2_main_kernel<{d}>" if dominant == "bwd_main" else f"fa_fwd_bf16_2tile_kernel<{d}>",
                      "bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_tf, 4), "traffic": traffic_val,
                      "algorithmic_bytes": nbytes[dominant],
@@ -411,6 +436,12 @@ def run_ours(args, rank, world, local):
         "clocks": clocks,
         "kernel_src": src_hash,
     }
+    if fwd_only is not None:
+        peak = float(load_peaks()[0]["bf16_tflops"])
+        out["fwd_only"] = {"launches": fwd_only["launches"], "ms": round(fwd_only["ms"], 4),
+                           "tflops": round(fwd_only["tflops"], 2),
+                           "pct_of_peak": round(100 * fwd_only["tflops"] / world / peak, 2),
+                           "clocks": fwd_only["clocks"]}
     if e2e is not None:
         out["e2e"] = {k: (round(v, 4) if isinstance(v, float) else v) for k, v in e2e.items()}
     if world == 1 and not args.no_cpu_baseline:
@@ -466,6 +497,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fwd-only", action="store_true", help="skip the separate forward-only timed region")
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d of a smaller case for profiling (default: the benchmark workload)")
     args = ap.parse_args(argv)
