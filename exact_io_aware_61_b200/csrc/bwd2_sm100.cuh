@@ -17,7 +17,9 @@
 //   warps 0-7   two compute warpgroups; warpgroup h owns query columns
 //               [64h, 64h + 64): P^T = exp2(S^T * scale * log2 e - LSE2) ->
 //               bf16 over its own S^T columns in TMEM, then
-//               dS^T = P^T (dP^T - D) scale -> shared memory (bf16)
+//               dS^T = P^T (dP^T - D) scale (bf16) -> TMEM, over the other
+//               half of those S^T columns (A operand of dK), and -> shared
+//               memory (operand of dQ)
 //   warps 8-11  dQ drain: the dQ tile leaves TMEM at once, then is added to
 //               the f32 accumulator with TMA tensor reduce-adds
 //   warp 12     TMA producer (K, V once; Q, LSE2, D double-buffered; dO)
@@ -26,6 +28,9 @@
 //   dP^T(t) [once dQ(t-1) left TMEM], dV += P^T dO, dK += dS^T Q,
 //   dQ(t) [into the dP^T columns], then S^T(t+1) at once, so the compute
 //   warpgroups start on step t+1 while the drain empties dQ(t).
+// Operand forms: an MMA whose A operand is in TMEM runs at the full rate,
+// one with both operands in shared memory is markedly slower, so dV and dK
+// take their A operand (P^T, dS^T) from TMEM.
 // TMEM: S^T / P^T at 0, dP^T / dQ at 128, dV at 256, dK at 256 + d.
 #pragma once
 
@@ -48,10 +53,12 @@ struct Bwd2Cfg {
       1024 + 2 * TILE + QST * QSTAGE_BYTES + DOST * TILE + DS_BYTES + DQ_STAGE_BYTES;
   static constexpr int THREADS = 512;
   // Launch with 128 registers per thread (16 warps, 4 per SM sub-partition),
-  // then redistribute per warpgroup: 128 x (120 + 120 + 168 + 104) = 512 x 128.
+  // then redistribute per warpgroup: 128 x (2 compute + drain + other) =
+  // 512 x 128. The drain holds a whole dQ row (HD registers), so at d = 64 it
+  // gives registers to the compute warpgroups.
   static constexpr int LAUNCH_REGS = 128;
-  static constexpr int COMPUTE_REGS = 120;
-  static constexpr int DRAIN_REGS = 168;
+  static constexpr int COMPUTE_REGS = HD == 64 ? 136 : 120;
+  static constexpr int DRAIN_REGS = HD == 64 ? 136 : 168;
   static constexpr int OTHER_REGS = 104;
   static_assert(128 * (2 * COMPUTE_REGS + DRAIN_REGS + OTHER_REGS) <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
@@ -210,7 +217,7 @@ __global__ void __launch_bounds__(512, 1)
   };
 
   if (warp >= 12) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
+    set_max_regs<C::OTHER_REGS, C::LAUNCH_REGS>();
     if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -287,12 +294,11 @@ __global__ void __launch_bounds__(512, 1)
         // dK += dS^T Q ; dQ = dS K
         if (!mbar_wait(smem_u32(&bar_dsfull), t & 1, wc)) break;
         tc_fence_after();
+        // (dS^T from TMEM: queries 64h + 32 .. of warpgroup h's columns)
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + C::T_DK, sdesc_sw128(sDS + off, 16, 1024), sdesc_sw128(qst + kk * 2048, 16384, 1024),
-                      id_kmn, (t > 0 || kk > 0));
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + C::T_DK, tmem + C::T_S + (kk >> 2) * 64 + 32 + (kk & 3) * 8,
+                      sdesc_sw128(qst + kk * 2048, 16384, 1024), id_kmn, (t > 0 || kk > 0));
         // dQ = dS K (M = queries, N = d)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -310,13 +316,14 @@ __global__ void __launch_bounds__(512, 1)
     }
     }  // warps 14, 15: idle
   } else if (warp < 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::COMPUTE_REGS));
+    set_max_regs<C::COMPUTE_REGS, C::LAUNCH_REGS>();
     // ---------------------------------------------------- compute warpgroups
     // Warpgroup `half` owns query columns [64 half, 64 half + 64) of every
     // step: it turns its S^T columns into P^T (bf16, written over its own
     // S^T columns 64 half .. 64 half + 31) and later its dP^T columns into
-    // dS^T (bf16, shared-memory block `half`). Both warpgroups cover all 128
-    // key rows (TMEM lane = key).
+    // dS^T (bf16, written over S^T columns 64 half + 32 .. 64 half + 63, and
+    // into shared-memory block `half`). Both warpgroups cover all 128 key
+    // rows (TMEM lane = key).
     const int half = warp >> 2;
     const int tid = threadIdx.x & 127;  // key row k0 + tid
     const int cb = half * 64;           // first query column of this warpgroup
@@ -388,6 +395,7 @@ __global__ void __launch_bounds__(512, 1)
           w[2 * x] = pack_bf16x2(e0, e1);
           w[2 * x + 1] = pack_bf16x2(e2, e3);
         }
+        tmem_st16(tmem + lane_base + C::T_S + cb + 32 + u * 16, w);
         // 32 queries = 64 bytes = four 16-byte chunks: chunk u*4 + v, swizzled by row
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -395,6 +403,7 @@ __global__ void __launch_bounds__(512, 1)
           *reinterpret_cast<uint4*>(ds_row + chunk * 16) = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(smem_u32(&bar_dsfull));
@@ -419,7 +428,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::DRAIN_REGS));
+    set_max_regs<C::DRAIN_REGS, C::LAUNCH_REGS>();
     // ------------------------------------------------------- dQ warpgroup
     // Thread tid holds query row q0 + tid of the dQ tile (TMEM lane = row).
     // The whole tile is loaded into registers and its columns released to

@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = tmem_slot;
 
   if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
+    set_max_regs<C::OTHER_REGS, C::LAUNCH_REGS>();
   }
   if (warp >= 10) {
     // idle warps of the third warpgroup
@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else {
     // ------------------------------------------------------------- softmax
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
+    set_max_regs<C::SOFTMAX_REGS, C::LAUNCH_REGS>();
     const int t = warp >> 2;                      // query tile of this warpgroup
     const int row = q0 + t * C::BM + (threadIdx.x & 127);
     const uint32_t lane_base = ((warp & 3) * 32u) << 16;

@@ -96,6 +96,19 @@ FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl& w) {
   return __all_sync(0xffffffffu, ok);
 }
 
+// Move this warp's register allocation from the launch count LAUNCH to N
+// (setmaxnreg: .inc to raise it, .dec to lower it). The caller's warpgroups
+// must add up to the launch allocation, or an .inc waits forever.
+template <int N, int LAUNCH>
+FA_DEV void set_max_regs() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg takes a multiple of 8 in [24, 256]");
+  if constexpr (N > LAUNCH) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+  } else if constexpr (N < LAUNCH) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+  }
+}
+
 // Named barrier over `count` threads (a multiple of 32), id 1..15.
 FA_DEV void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
