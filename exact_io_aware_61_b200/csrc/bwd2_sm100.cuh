@@ -12,8 +12,12 @@
 //   dP = dO V^T                     D  = rowsum(dO * O)   (prep kernel)
 //   dS = P * (dP - D)               dQ = scale dS K,  dK = scale dS^T Q
 //
-// One CTA per (128-key tile, batch, KV head); it loops over the query heads
-// of the group and the query tiles that see its key tile. Roles (16 warps):
+// One CTA per (128-key tile, batch, KV head, head slice); it loops over its
+// slice of the query heads of the group and the query tiles that see its key
+// tile. With one slice (the usual case) it writes dK and dV in bf16; when the
+// host splits the group over several CTAs (too few CTAs for the SMs
+// otherwise, as with one KV head), each CTA adds its f32 share into dK/dV
+// accumulators that a conversion kernel rounds afterwards. Roles (16 warps):
 //   warps 0-7   two compute warpgroups; warpgroup h owns query columns
 //               [64h, 64h + 64): P^T = exp2(S^T * scale * log2 e - LSE2) ->
 //               bf16 over its own S^T columns in TMEM, then
@@ -75,7 +79,10 @@ struct Bwd2Params {
   float* dq_acc;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* dk_acc;   // [B*Hkv][N][d] f32, used when head_split > 1
+  float* dv_acc;
   int N, Npad, Hq, Hkv, num_tiles;
+  int head_split;  // CTAs sharing the query heads of one (KV head, key tile)
   float scale_log2;
   float scale;
   int causal;
@@ -169,15 +176,20 @@ __global__ void __launch_bounds__(512, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int bhkv = static_cast<int>(blockIdx.x) / p.num_tiles;
-  const int kt = static_cast<int>(blockIdx.x) - bhkv * p.num_tiles;  // tile 0 has the most work when causal
+  const int per_kv = p.num_tiles * p.head_split;
+  const int bhkv = static_cast<int>(blockIdx.x) / per_kv;
+  const int rem = static_cast<int>(blockIdx.x) - bhkv * per_kv;
+  const int kt = rem / p.head_split;  // tile 0 has the most work when causal
+  const int slice = rem - kt * p.head_split;
   const int k0 = kt * 128;
   const int b = bhkv / p.Hkv;
   const int hkv = bhkv - b * p.Hkv;
   const int group = p.Hq / p.Hkv;
+  const int heads = group / p.head_split;  // query heads of this CTA's slice
+  const int h_first = slice * heads;
   const int i_begin = p.causal ? kt : 0;
   const int per_head = p.num_tiles - i_begin;
-  const int steps = group * per_head;
+  const int steps = heads * per_head;
 
   WaitCtl wc{&abort_flag, p.timeout_ns};
 
@@ -213,7 +225,7 @@ __global__ void __launch_bounds__(512, 1)
   auto step_tile = [&](int t, int& bhq, int& q0) {
     const int hh = t / per_head;
     q0 = (i_begin + (t - hh * per_head)) * 128;
-    bhq = b * p.Hq + hkv * group + hh;
+    bhq = b * p.Hq + hkv * group + h_first + hh;
   };
 
   if (warp >= 12) {
@@ -408,22 +420,35 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_before();
       mbar_arrive(smem_u32(&bar_dsfull));
     }
-    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (dS carries the scale)
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (dS carries the
+    // scale): bf16 rows, or, when the group's heads are split over several
+    // CTAs, f32 rows added into the accumulators
     if (ok && warp_wait(smem_u32(&bar_final), 0, wc)) {
       tc_fence_after();
-      __nv_bfloat16* out = (half == 0 ? p.dv : p.dk) + (static_cast<size_t>(bhkv) * p.N + (key_live ? key : 0)) * HD;
+      const size_t row_off = (static_cast<size_t>(bhkv) * p.N + (key_live ? key : 0)) * HD;
+      __nv_bfloat16* out = (half == 0 ? p.dv : p.dk) + row_off;
+      float* acc = p.head_split > 1 ? (half == 0 ? p.dv_acc : p.dk_acc) + row_off : nullptr;
       const uint32_t col = half == 0 ? C::T_DV : C::T_DK;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_base + col + c * 32, r);
-        uint4 w[4];
-        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+        if (p.head_split > 1) {
+          if (key_live) {
 #pragma unroll
-        for (int x = 0; x < 16; ++x) wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]), __uint_as_float(r[2 * x + 1]));
-        if (key_live) {
+            for (int x = 0; x < 8; ++x)
+              red_add_v4_f32(acc + c * 32 + 4 * x, __uint_as_float(r[4 * x]), __uint_as_float(r[4 * x + 1]),
+                             __uint_as_float(r[4 * x + 2]), __uint_as_float(r[4 * x + 3]));
+          }
+        } else {
+          uint4 w[4];
+          uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-          for (int x = 0; x < 4; ++x) reinterpret_cast<uint4*>(out + c * 32)[x] = w[x];
+          for (int x = 0; x < 16; ++x) wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]), __uint_as_float(r[2 * x + 1]));
+          if (key_live) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) reinterpret_cast<uint4*>(out + c * 32)[x] = w[x];
+          }
         }
       }
     }

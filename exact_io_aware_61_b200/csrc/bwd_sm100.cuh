@@ -4,7 +4,9 @@
 //                        128-row-padded workspace rows (+inf / 0 in the
 //                        padding, so padded queries get zero weight), and
 //                        zeroing of the f32 dQ accumulator
-//   fa_bwd_dq_kernel     f32 dQ accumulator -> bf16 dQ
+//   fa_bwd_dq_kernel     f32 accumulator -> bf16 (dQ; dK, dV when the
+//                        backward splits a group's heads over CTAs)
+//   fa_zero_f32_kernel   zero an f32 accumulator
 #pragma once
 
 #include <cuda.h>
@@ -78,6 +80,13 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict_
     w.y = pack_bf16x2(v.z, v.w);
     reinterpret_cast<uint2*>(dq)[i] = w;
   }
+}
+
+// Grid-stride zeroing of n4 float4s.
+__global__ void __launch_bounds__(256) fa_zero_f32_kernel(float* __restrict__ p, size_t n4) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    reinterpret_cast<float4*>(p)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 }  // namespace fa

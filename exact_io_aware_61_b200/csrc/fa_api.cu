@@ -244,27 +244,65 @@ int launch_fwd_f32(const void* q, const void* k, const void* v, void* o, float* 
 
 size_t padded_rows(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 
-// Workspace carve-up: D [B*Hq][Npad], LSE*log2(e) [B*Hq][Npad], dQ accumulator [B*Hq][N][d], all f32.
+// How many CTAs share the query heads of one (KV head, 128-key tile) in the
+// backward: 1 unless B * Hkv * (key tiles) is below 592 (4 CTAs per SM of a
+// 148-SM part), then the smallest divisor of the group size that reaches it,
+// or the group size. A pure function of the shape, so the workspace size
+// does not depend on the device.
+int bwd_head_split(int B, int Hq, int Hkv, int N) {
+  const long long ctas = static_cast<long long>(B) * Hkv * static_cast<long long>(padded_rows(N) / 128);
+  const int g = Hq / Hkv;
+  for (int s = 1; s <= g; ++s)
+    if (g % s == 0 && ctas * s >= 592) return s;
+  return g;
+}
+
+// Workspace carve-up, all f32: D [B*Hq][Npad], LSE*log2(e) [B*Hq][Npad],
+// dQ accumulator [B*Hq][N][d]; when the backward splits a group's heads over
+// CTAs, also dK and dV accumulators [B*Hkv][N][d].
 struct BwdWorkspace {
   float* delta;
   float* lse2;
   float* dq_acc;
+  float* dk_acc;  // null without a split
+  float* dv_acc;
 };
 
-BwdWorkspace carve(void* ws, int B, int Hq, int N) {
+BwdWorkspace carve(void* ws, int B, int Hq, int Hkv, int N, int d) {
   const size_t npad = padded_rows(N);
   const size_t rows_q = static_cast<size_t>(B) * Hq;
+  const size_t kv_elems = static_cast<size_t>(B) * Hkv * static_cast<size_t>(N) * d;
   BwdWorkspace w;
   w.delta = static_cast<float*>(ws);
   w.lse2 = w.delta + rows_q * npad;
   w.dq_acc = w.lse2 + rows_q * npad;
+  const bool split = bwd_head_split(B, Hq, Hkv, N) > 1;
+  w.dk_acc = split ? w.dq_acc + rows_q * static_cast<size_t>(N) * d : nullptr;
+  w.dv_acc = split ? w.dk_acc + kv_elems : nullptr;
   return w;
 }
 
+// f32 -> bf16 rounding of n elements (a multiple of 4) on `stream`.
+int launch_convert(const float* acc, void* out, size_t n, cudaStream_t stream) {
+  const size_t n4 = n / 4;
+  const size_t want = (n4 + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
+  fa::fa_bwd_dq_kernel<<<grid, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16*>(out), n4);
+  return launch_status();
+}
+
+int launch_zero(float* p, size_t n, cudaStream_t stream) {
+  const size_t n4 = n / 4;
+  const size_t want = (n4 + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
+  fa::fa_zero_f32_kernel<<<grid, 256, 0, stream>>>(p, n4);
+  return launch_status();
+}
+
 template <int HD>
-int launch_bwd_prep(const void* o, const float* lse, const void* dO, void* ws, int B, int Hq, int N,
+int launch_bwd_prep(const void* o, const float* lse, const void* dO, void* ws, int B, int Hq, int Hkv, int N,
                     cudaStream_t stream) {
-  const BwdWorkspace w = carve(ws, B, Hq, N);
+  const BwdWorkspace w = carve(ws, B, Hq, Hkv, N, HD);
   const size_t npad = padded_rows(N);
   fa::BwdPrepParams pp;
   pp.o = static_cast<const __nv_bfloat16*>(o);
@@ -285,7 +323,9 @@ template <int HD>
 int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* ws,
                     int B, int Hq, int Hkv, int N, float scale, int causal, cudaStream_t stream) {
   using C = fa::Bwd2Cfg<HD>;
-  const BwdWorkspace w = carve(ws, B, Hq, N);
+  const BwdWorkspace w = carve(ws, B, Hq, Hkv, N, HD);
+  const int split = bwd_head_split(B, Hq, Hkv, N);
+  const size_t kv_elems = static_cast<size_t>(B) * Hkv * static_cast<size_t>(N) * HD;
   const size_t npad = padded_rows(N);
   const uint64_t rows_q = static_cast<uint64_t>(B) * Hq, rows_kv = static_cast<uint64_t>(B) * Hkv;
   CUtensorMap mq, mk, mv, mdo, mdq;
@@ -301,6 +341,9 @@ int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO,
   p.dq_acc = w.dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dk_acc = w.dk_acc;
+  p.dv_acc = w.dv_acc;
+  p.head_split = split;
   p.N = N;
   p.Npad = static_cast<int>(npad);
   p.Hq = Hq;
@@ -310,7 +353,7 @@ int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO,
   p.scale = scale;
   p.causal = causal;
   p.timeout_ns = timeout_now();
-  const long long blocks = static_cast<long long>(p.num_tiles) * B * Hkv;
+  const long long blocks = static_cast<long long>(p.num_tiles) * B * Hkv * split;
   if (blocks > INT32_MAX) return FA_ERR_INVALID;
   // The kernel redistributes registers between warpgroups (setmaxnreg) on
   // the assumption of exactly LAUNCH_REGS per thread at launch.
@@ -322,18 +365,22 @@ int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO,
                                 C::LAUNCH_REGS);
     return FA_ERR_UNSUPPORTED;
   }
+  if (split > 1) {
+    if ((rc = launch_zero(w.dk_acc, 2 * kv_elems, stream)) != FA_OK) return rc;  // dK and dV accumulators
+  }
   fa::fa_bwd2_main_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
                                                                                                      mdq, p);
-  return launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>));
+  if ((rc = launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>))) != FA_OK) return rc;
+  if (split > 1) {
+    if ((rc = launch_convert(w.dk_acc, dk, kv_elems, stream)) != FA_OK) return rc;
+    if ((rc = launch_convert(w.dv_acc, dv, kv_elems, stream)) != FA_OK) return rc;
+  }
+  return FA_OK;
 }
 
-int launch_bwd_dq(void* dq, void* ws, int B, int Hq, int N, int d, cudaStream_t stream) {
-  const BwdWorkspace w = carve(ws, B, Hq, N);
-  const size_t n4 = static_cast<size_t>(B) * Hq * static_cast<size_t>(N) * d / 4;
-  const size_t want = (n4 + 255) / 256;
-  const unsigned grid = static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
-  fa::fa_bwd_dq_kernel<<<grid, 256, 0, stream>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), n4);
-  return launch_status();
+int launch_bwd_dq(void* dq, void* ws, int B, int Hq, int Hkv, int N, int d, cudaStream_t stream) {
+  const BwdWorkspace w = carve(ws, B, Hq, Hkv, N, d);
+  return launch_convert(w.dq_acc, dq, static_cast<size_t>(B) * Hq * static_cast<size_t>(N) * d, stream);
 }
 
 // Checks shared by the backward entry points. `ptrs` must all be 16-byte aligned and non-null.
@@ -398,7 +445,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || d < 1 || Hq % Hkv != 0) return 0;
   const size_t rows_q = static_cast<size_t>(B) * Hq;
-  return sizeof(float) * (2 * rows_q * padded_rows(N) + rows_q * static_cast<size_t>(N) * d);
+  const size_t kv_acc = bwd_head_split(B, Hq, Hkv, N) > 1 ? 2 * static_cast<size_t>(B) * Hkv * N * d : 0;
+  return sizeof(float) * (2 * rows_q * padded_rows(N) + rows_q * static_cast<size_t>(N) * d + kv_acc);
 }
 
 int fa_bwd_prep(const void* o, const float* lse, const void* dO, void* workspace, size_t workspace_bytes, int B,
@@ -407,8 +455,8 @@ int fa_bwd_prep(const void* o, const float* lse, const void* dO, void* workspace
   int rc = check_bwd({o, lse, dO}, workspace, workspace_bytes, B, Hq, Hkv, N, d, 1.0f, 0, dtype, &dev);
   if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd_prep<64>(o, lse, dO, workspace, B, Hq, N, s)
-                 : launch_bwd_prep<128>(o, lse, dO, workspace, B, Hq, N, s);
+  return d == 64 ? launch_bwd_prep<64>(o, lse, dO, workspace, B, Hq, Hkv, N, s)
+                 : launch_bwd_prep<128>(o, lse, dO, workspace, B, Hq, Hkv, N, s);
 }
 
 int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* workspace,
@@ -427,7 +475,7 @@ int fa_bwd_dq(void* dq, void* workspace, size_t workspace_bytes, int B, int Hq, 
   int dev = 0;
   int rc = check_bwd({dq}, workspace, workspace_bytes, B, Hq, Hkv, N, d, 1.0f, 0, dtype, &dev);
   if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
-  return launch_bwd_dq(dq, workspace, B, Hq, N, d, reinterpret_cast<cudaStream_t>(stream));
+  return launch_bwd_dq(dq, workspace, B, Hq, Hkv, N, d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
@@ -439,15 +487,15 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) {
-    if ((rc = launch_bwd_prep<64>(o, lse, dO, workspace, B, Hq, N, s)) != FA_OK) return rc;
+    if ((rc = launch_bwd_prep<64>(o, lse, dO, workspace, B, Hq, Hkv, N, s)) != FA_OK) return rc;
     if ((rc = launch_bwd_main<64>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
       return rc;
   } else {
-    if ((rc = launch_bwd_prep<128>(o, lse, dO, workspace, B, Hq, N, s)) != FA_OK) return rc;
+    if ((rc = launch_bwd_prep<128>(o, lse, dO, workspace, B, Hq, Hkv, N, s)) != FA_OK) return rc;
     if ((rc = launch_bwd_main<128>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
       return rc;
   }
-  return launch_bwd_dq(dq, workspace, B, Hq, N, d, s);
+  return launch_bwd_dq(dq, workspace, B, Hq, Hkv, N, d, s);
 }
 
 }  // extern "C"
@@ -503,20 +551,21 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   rc = check_bwd({q, k, v, o, lse, dO, dq, dk, dv}, scratch, kNoAllocScratchBytes, B, Hq, Hkv, N, d, scale, causal,
                  dtype, &dev);
   if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
-  // The prep kernel rewrites every scratch byte this problem reads (D, LSE,
-  // and the dQ accumulator, which it zeroes), so what an earlier call left
-  // in the array does not matter.
+  // Every scratch byte this problem reads is rewritten first (D, LSE and the
+  // dQ accumulator by the prep kernel; the dK/dV accumulators, when the
+  // group's heads are split, by a zeroing kernel before the main kernel), so
+  // what an earlier call left in the array does not matter.
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) {
-    if ((rc = launch_bwd_prep<64>(o, lse, dO, scratch, B, Hq, N, s)) != FA_OK) return rc;
+    if ((rc = launch_bwd_prep<64>(o, lse, dO, scratch, B, Hq, Hkv, N, s)) != FA_OK) return rc;
     if ((rc = launch_bwd_main<64>(q, k, v, dO, dk, dv, scratch, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
       return rc;
   } else {
-    if ((rc = launch_bwd_prep<128>(o, lse, dO, scratch, B, Hq, N, s)) != FA_OK) return rc;
+    if ((rc = launch_bwd_prep<128>(o, lse, dO, scratch, B, Hq, Hkv, N, s)) != FA_OK) return rc;
     if ((rc = launch_bwd_main<128>(q, k, v, dO, dk, dv, scratch, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
       return rc;
   }
-  return launch_bwd_dq(dq, scratch, B, Hq, N, d, s);
+  return launch_bwd_dq(dq, scratch, B, Hq, Hkv, N, d, s);
 }
 
 int fa_last_device_status(fa_stream_t stream) {

@@ -96,6 +96,12 @@ FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl& w) {
   return __all_sync(0xffffffffu, ok);
 }
 
+// Atomic add of four consecutive floats (16-byte aligned) in global memory.
+FA_DEV void red_add_v4_f32(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 // Move this warp's register allocation from the launch count LAUNCH to N
 // (setmaxnreg: .inc to raise it, .dec to lower it). The caller's warpgroups
 // must add up to the launch allocation, or an .inc waits forever.

@@ -99,8 +99,11 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs: the
  * per-row term D = rowsum(dO * O) and the log2-scaled LSE, both float32 and
  * padded to a multiple of 128 rows per head, plus a float32 dQ accumulator
- * [B][Hq][N][d]. Linear in N: nothing N x N is ever allocated. Returns 0 for
- * invalid sizes.
+ * [B][Hq][N][d]. When B * Hkv * ceil(N / 128) < 592, the backward splits
+ * each group's query heads over several CTAs (the smallest divisor s of
+ * Hq / Hkv with that product times s >= 592, else Hq / Hkv) and the
+ * workspace also holds float32 dK and dV accumulators [B][Hkv][N][d]. Linear
+ * in N: nothing N x N is ever allocated. Returns 0 for invalid sizes.
  */
 FA_API size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
 
@@ -122,7 +125,9 @@ FA_API size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
  * dK = scale dS^T Q. Supports dtype FA_BF16 with d in {64, 128}; other
  * combinations return FA_ERR_UNSUPPORTED. Three kernels run in stream order:
  * D and LSE preparation (and zeroing of the dQ accumulator), the main
- * recompute kernel, and the dQ conversion.
+ * recompute kernel, and the dQ conversion; with split query heads (see
+ * fa_bwd_workspace_size) the main stage also zeroes the dK/dV accumulators
+ * before, and rounds them to dk, dv after, its kernel.
  */
 FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o,
            const float* lse, const void* dO, void* dq, void* dk, void* dv,
@@ -142,8 +147,9 @@ FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o,
  *   Reads o, lse, dO.
  * fa_bwd_main -- the recompute kernel: per 128-key tile of each KV head it
  *   rebuilds P from Q, K and the padded LSE, and forms dV, dP, dS, dK (written
- *   to dk, dv) and adds each dQ tile into the accumulator. Needs fa_bwd_prep
- *   to have run on the same workspace.
+ *   to dk, dv, through f32 accumulators when the query heads are split) and
+ *   adds each dQ tile into the accumulator. Needs fa_bwd_prep to have run on
+ *   the same workspace.
  * fa_bwd_dq -- converts the f32 dQ accumulator to dq (bf16).
  */
 FA_API int fa_bwd_prep(const void* o, const float* lse, const void* dO,

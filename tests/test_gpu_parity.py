@@ -190,6 +190,49 @@ def test_bwd_train_causal_b2_h16_n4096_d128(fa):
             assert err <= GRAD_TOL, (name, b, h, err)
 
 
+def test_bwd_gqa_causal_b1_h8_kv2_n4096_d128_full_group(fa):
+    """GQA backward against the full oracle on one KV head and its whole group
+    (dK and dV of a KV head sum over the group's four query heads)."""
+    B, Hq, Hkv, N, d = 1, 8, 2, 4096, 128
+    inp = INP.make_inputs(B, Hq, Hkv, N, d, "bf16", seed=4096 + 8, grad=True)
+    dq, dk, dv = _run_bwd(fa, inp, True, d ** -0.5)
+    g = Hq // Hkv
+    for hk in range(Hkv):
+        qs, kvs = slice(hk * g, (hk + 1) * g), slice(hk, hk + 1)
+        rq, rk, rv, _ = ORACLE.attention_backward(INP.as_f64(inp["q"][:, qs]), INP.as_f64(inp["k"][:, kvs]),
+                                                 INP.as_f64(inp["v"][:, kvs]), INP.as_f64(inp["do"][:, qs]),
+                                                 d ** -0.5, True)
+        for name, got, ref in (("dq", dq[:, qs], rq), ("dk", dk[:, kvs], rk), ("dv", dv[:, kvs], rv)):
+            err = _rel_fro(INP.as_f64(got), ref)
+            assert err <= GRAD_TOL, (name, hk, err)
+
+
+def test_bwd_gqa_causal_b1_h32_kv8_n16384_d128(fa):
+    """GQA backward at the 16k-token GQA workload: exact dQ on sampled rows of
+    every query head, and for every KV head the identity sum_j dV_j =
+    sum over the group's heads of sum_i dO_i (each row of P sums to one)."""
+    w = INP.WORKLOADS["gqa_causal_bf16_b1_h32_kv8_n16384_d128"]
+    inp = INP.make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, "bf16", seed=16384 + 32, grad=True)
+    dq, dk, dv = _run_bwd(fa, inp, True, w.scale)
+    dq_h = dq.float().cpu().numpy()
+    dv_h = dv.float().cpu().numpy().astype(np.float64)
+    q, k, v, do = (inp[n].float().numpy() for n in ("q", "k", "v", "do"))
+    g = w.Hq // w.Hkv
+    for hk in range(w.Hkv):
+        lhs = dv_h[0, hk].sum(axis=0)
+        rhs = do[0, hk * g:(hk + 1) * g].astype(np.float64).sum(axis=(0, 1))
+        assert _rel_fro(lhs, rhs) <= GRAD_TOL, ("dv sum", hk)
+    rng = np.random.default_rng(11)
+    worst = 0.0
+    for h in range(w.Hq):
+        rows = _sample_rows(w.N, rng, n_random=6)
+        rq, _, _ = ORACLE.attention_backward_rows(q, k, v, do, w.scale, True, 0, h, rows)
+        worst = max(worst, _rel_fro(dq_h[0, h, rows].astype(np.float64), rq))
+    assert worst <= GRAD_TOL, worst
+    assert np.all(np.isfinite(dq_h)) and np.all(np.isfinite(dv_h))
+    assert torch.isfinite(dk.float()).all()
+
+
 # ---------------------------------------------------------- ABI behaviour
 
 def test_abi_rejects_bad_arguments_without_writing(fa):
