@@ -66,6 +66,7 @@ struct Bwd2Cfg {
   static constexpr int OTHER_REGS = 104;
   static_assert(128 * (2 * COMPUTE_REGS + DRAIN_REGS + OTHER_REGS) <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
+  static constexpr int KV_GROUP = 8;  // (batch, KV head) pairs scheduled together
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0;
   static constexpr uint32_t T_DP = 128;
@@ -83,6 +84,7 @@ struct Bwd2Params {
   float* dv_acc;
   int N, Npad, Hq, Hkv, num_tiles;
   int head_split;  // CTAs sharing the query heads of one (KV head, key tile)
+  int BHkv;        // B * Hkv
   float scale_log2;
   float scale;
   int causal;
@@ -176,11 +178,18 @@ __global__ void __launch_bounds__(512, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // Block order: groups of KV_GROUP (batch, KV head) pairs, whose K, V, Q and
+  // dO stay in L2 together; inside a group the key tiles go heaviest first
+  // (tile 0 has the most work when causal), each over the group's heads and
+  // head slices, so the last blocks to start are the shortest.
   const int per_kv = p.num_tiles * p.head_split;
-  const int bhkv = static_cast<int>(blockIdx.x) / per_kv;
-  const int rem = static_cast<int>(blockIdx.x) - bhkv * per_kv;
-  const int kt = rem / p.head_split;  // tile 0 has the most work when causal
-  const int slice = rem - kt * p.head_split;
+  const int grp = static_cast<int>(blockIdx.x) / (C::KV_GROUP * per_kv);
+  const int in_grp = min(C::KV_GROUP, p.BHkv - grp * C::KV_GROUP);
+  const int r0 = static_cast<int>(blockIdx.x) - grp * C::KV_GROUP * per_kv;
+  const int kt = r0 / (in_grp * p.head_split);
+  const int r1 = r0 - kt * in_grp * p.head_split;
+  const int bhkv = grp * C::KV_GROUP + r1 / p.head_split;
+  const int slice = r1 - (r1 / p.head_split) * p.head_split;
   const int k0 = kt * 128;
   const int b = bhkv / p.Hkv;
   const int hkv = bhkv - b * p.Hkv;

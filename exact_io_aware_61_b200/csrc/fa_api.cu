@@ -344,6 +344,7 @@ int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO,
   p.dk_acc = w.dk_acc;
   p.dv_acc = w.dv_acc;
   p.head_split = split;
+  p.BHkv = B * Hkv;
   p.N = N;
   p.Npad = static_cast<int>(npad);
   p.Hq = Hq;
