@@ -30,10 +30,13 @@ template <int HD>
 struct Fwd2Cfg {
   static constexpr int BM = 128;  // rows per query tile
   static constexpr int BN = 128;  // keys per key tile
-  static constexpr int STAGES = HD == 64 ? 4 : 2;
+  // K and V ring depths. K runs one tile ahead of V (S(j+1) is issued right
+  // after P(j)V(j)), so at d = 128 it gets the extra stage that fits.
+  static constexpr int KST = HD == 64 ? 4 : 3;
+  static constexpr int VST = HD == 64 ? 4 : 2;
   static constexpr int Q_TILE_BYTES = BM * HD * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
-  static constexpr int SMEM_BYTES = 1024 + 2 * Q_TILE_BYTES + 2 * STAGES * KV_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + 2 * Q_TILE_BYTES + (KST + VST) * KV_BYTES;
   static constexpr int THREADS = 384;
   static constexpr int LAUNCH_REGS = 168;  // the split below assumes exactly this
   static constexpr int SOFTMAX_REGS = 216;
@@ -132,11 +135,11 @@ __global__ void __launch_bounds__(384, 1)
     fa_fwd_bf16_2tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const Fwd2Params p) {
   using C = Fwd2Cfg<HD>;
-  constexpr int ST = C::STAGES;
+  constexpr int KST = C::KST, VST = C::VST;
   constexpr int KCH = HD / 64;
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_kfull[ST], bar_kempty[ST], bar_vfull[ST], bar_vempty[ST];
+  __shared__ uint64_t bar_q, bar_kfull[KST], bar_kempty[KST], bar_vfull[VST], bar_vempty[VST];
   __shared__ uint64_t bar_sfull[2], bar_pfull[2], bar_odone[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sQ = base;  // tile t at sQ + t * Q_TILE_BYTES
   const uint32_t sK = sQ + 2 * C::Q_TILE_BYTES;
-  const uint32_t sV = sK + ST * C::KV_BYTES;
+  const uint32_t sV = sK + KST * C::KV_BYTES;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -176,9 +179,11 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(smem_u32(&bar_q), 1);
-    for (int s = 0; s < ST; ++s) {
+    for (int s = 0; s < KST; ++s) {
       mbar_init(smem_u32(&bar_kfull[s]), 1);
       mbar_init(smem_u32(&bar_kempty[s]), 1);
+    }
+    for (int s = 0; s < VST; ++s) {
       mbar_init(smem_u32(&bar_vfull[s]), 1);
       mbar_init(smem_u32(&bar_vempty[s]), 1);
     }
@@ -215,19 +220,24 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < KCH; ++c)
           tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * (C::BM * 128), &tm_q, smem_u32(&bar_q), c * 64,
                       q0 + t * C::BM, bh);
-      for (int j = 0; j < n_max; ++j) {
-        const int s = j % ST;
-        const uint32_t ph = (j / ST) & 1;
-        if (!mbar_wait(smem_u32(&bar_kempty[s]), ph ^ 1, wc)) break;
-        mbar_arrive_expect_tx(smem_u32(&bar_kfull[s]), C::KV_BYTES);
-        for (int c = 0; c < KCH; ++c)
-          tma_load_3d(sK + s * C::KV_BYTES + c * (C::BN * 128), &tm_k, smem_u32(&bar_kfull[s]), c * 64,
-                      j * C::BN, bh_kv);
-        if (!mbar_wait(smem_u32(&bar_vempty[s]), ph ^ 1, wc)) break;
-        mbar_arrive_expect_tx(smem_u32(&bar_vfull[s]), C::KV_BYTES);
-        for (int c = 0; c < KCH; ++c)
-          tma_load_3d(sV + s * C::KV_BYTES + c * (C::BN * 128), &tm_v, smem_u32(&bar_vfull[s]), c * 64,
-                      j * C::BN, bh_kv);
+      // order K(0), K(1), V(0), K(2), V(1), ...: K one tile ahead of V
+      for (int i = 0; i <= n_max; ++i) {
+        if (i < n_max) {
+          const int s = i % KST;
+          if (!mbar_wait(smem_u32(&bar_kempty[s]), ((i / KST) & 1) ^ 1, wc)) break;
+          mbar_arrive_expect_tx(smem_u32(&bar_kfull[s]), C::KV_BYTES);
+          for (int c = 0; c < KCH; ++c)
+            tma_load_3d(sK + s * C::KV_BYTES + c * (C::BN * 128), &tm_k, smem_u32(&bar_kfull[s]), c * 64,
+                        i * C::BN, bh_kv);
+        }
+        if (i >= 1) {
+          const int j = i - 1, s = j % VST;
+          if (!mbar_wait(smem_u32(&bar_vempty[s]), ((j / VST) & 1) ^ 1, wc)) break;
+          mbar_arrive_expect_tx(smem_u32(&bar_vfull[s]), C::KV_BYTES);
+          for (int c = 0; c < KCH; ++c)
+            tma_load_3d(sV + s * C::KV_BYTES + c * (C::BN * 128), &tm_v, smem_u32(&bar_vfull[s]), c * 64,
+                        j * C::BN, bh_kv);
+        }
       }
     }
   } else if (warp == 9) {
@@ -236,7 +246,7 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, HD, false, true);
       auto issue_s = [&](int t, int j) {
-        const uint32_t kb = sK + (j % ST) * C::KV_BYTES;
+        const uint32_t kb = sK + (j % KST) * C::KV_BYTES;
         const uint32_t qb = sQ + t * C::Q_TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
@@ -254,13 +264,13 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(smem_u32(&bar_kempty[0]));
       }
       for (int j = 0; ok && j < n_max; ++j) {
-        const int s = j % ST;
+        const int s = j % VST;
         bool v_ready = false, k_next_ready = false;
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= n_t[t]) continue;
           if (!mbar_wait(smem_u32(&bar_pfull[t]), j & 1, wc)) { ok = false; break; }
           if (!v_ready) {
-            if (!mbar_wait(smem_u32(&bar_vfull[s]), (j / ST) & 1, wc)) { ok = false; break; }
+            if (!mbar_wait(smem_u32(&bar_vfull[s]), (j / VST) & 1, wc)) { ok = false; break; }
             v_ready = true;
           }
           tc_fence_after();
@@ -272,7 +282,7 @@ __global__ void __launch_bounds__(384, 1)
           mma_commit(smem_u32(&bar_odone[t]));
           if (j + 1 < n_t[t]) {
             if (!k_next_ready) {
-              if (!mbar_wait(smem_u32(&bar_kfull[(j + 1) % ST]), ((j + 1) / ST) & 1, wc)) { ok = false; break; }
+              if (!mbar_wait(smem_u32(&bar_kfull[(j + 1) % KST]), ((j + 1) / KST) & 1, wc)) { ok = false; break; }
               k_next_ready = true;
               tc_fence_after();
             }
@@ -281,7 +291,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         mma_commit(smem_u32(&bar_vempty[s]));
-        if (k_next_ready) mma_commit(smem_u32(&bar_kempty[(j + 1) % ST]));
+        if (k_next_ready) mma_commit(smem_u32(&bar_kempty[(j + 1) % KST]));
       }
     }
   } else {
