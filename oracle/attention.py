@@ -41,6 +41,17 @@ KV head ``h // (Hq // Hkv)``; dK and dV sum over the query heads of a group.
 A row with no visible key (impossible for the square causal mask, kept for
 completeness) gets ``O = 0`` and ``LSE = -inf``.
 
+Queries against a longer key sequence (a KV cache: ``Nq`` new queries, ``Nk``
+cached keys that include them). The pages name the KV cache as what now
+limits serving (fanfani.net, section "The backward pass, and where the memory
+saving comes from"; synthetic.wiki, section "Where to be careful") without a
+formula; the reading taken here is the usual one: the queries are the last ``Nq`` positions, so query ``i`` sits at
+position ``Nk - Nq + i`` and, under the causal mask, sees keys ``j <= Nk - Nq
++ i``. ``merge_partial_states`` combines softmax states of disjoint key sets
+with the rescale rule of fanfani.net, section "A pinch of math: making the
+softmax work in pieces" (the same rule that carries the running state from one
+key block to the next).
+
 Layouts: Q, O, dO, dQ are ``[B, Hq, N, d]``; K, V, dK, dV are
 ``[B, Hkv, N, d]``; LSE and D are ``[B, Hq, N]``. All arithmetic is float64.
 """
@@ -60,6 +71,9 @@ __all__ = [
     "attention_backward",
     "attention_backward_rows",
     "score_matrix_bytes",
+    "attention_forward_kvcache",
+    "partial_state",
+    "merge_partial_states",
 ]
 
 
@@ -282,3 +296,61 @@ def score_gradient(p, dp, D):
 def score_matrix_bytes(N: int, heads: int, bytes_per_element: int) -> int:
     """Bytes the unfused path would need to hold the N x N scores of ``heads`` heads."""
     return N * N * heads * bytes_per_element
+
+
+def attention_forward_kvcache(q, k, v, scale: float, causal: bool):
+    """Exact attention of ``Nq`` queries against ``Nk >= Nq`` keys.
+
+    ``q`` is ``[B, Hq, Nq, d]``, ``k`` and ``v`` are ``[B, Hkv, Nk, d]``. Query
+    ``i`` is at position ``Nk - Nq + i``; with ``causal`` it sees the keys at
+    positions up to its own. Returns ``(O [B,Hq,Nq,d], LSE [B,Hq,Nq])``.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    B, Hq, Nq, _ = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if Nq > Nk:
+        raise ValueError("a KV cache holds at least the queries' own positions")
+    pos = Nk - Nq + np.arange(Nq)
+    o = np.empty((B, Hq, Nq, v.shape[-1]))
+    lse = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            hk = kv_head_of(h, Hq, Hkv)
+            p, m, l = softmax_rows(masked_scores(q[b, h], k[b, hk], scale, causal, rows=pos))
+            o[b, h] = p @ v[b, hk]
+            lse[b, h] = _lse(m, l)
+    return o, lse
+
+
+def partial_state(s, v):
+    """Softmax state of one set of keys: ``(m, l, o)`` per query row.
+
+    ``s`` holds the (masked) scaled scores ``[rows, keys]`` of the set and ``v``
+    its values ``[keys, d]``: ``m`` is the row maximum, ``l = sum exp(s - m)``
+    and ``o = sum exp(s - m) v`` (not divided by ``l``). A row with every key
+    masked has ``m = -inf``, ``l = 0``, ``o = 0``.
+    """
+    p, m, l = softmax_rows(_f64(s))
+    return m, l, (p * l[:, None]) @ _f64(v)
+
+
+def merge_partial_states(ms, ls, os):
+    """Combine softmax states of disjoint key sets into ``(O, LSE)``.
+
+    ``ms``, ``ls`` are ``[sets, rows]`` and ``os`` is ``[sets, rows, d]``, each
+    set's state as :func:`partial_state` gives it. With ``M = max_s m_s``, the
+    states are rescaled by ``exp(m_s - M)`` and added: ``L = sum_s l_s
+    exp(m_s - M)``, ``o = sum_s o_s exp(m_s - M)``; then ``O = o / L`` and
+    ``LSE = M + ln L``.
+    """
+    ms, ls, os = _f64(ms), _f64(ls), _f64(os)
+    M = np.max(ms, axis=0)
+    M_safe = np.where(np.isfinite(M), M, 0.0)
+    w = np.where(np.isfinite(ms), np.exp(ms - M_safe[None, :]), 0.0)
+    L = np.sum(w * ls, axis=0)
+    o = np.sum(w[:, :, None] * os, axis=0)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = np.where(L[:, None] > 0, o / np.where(L > 0, L, 1.0)[:, None], 0.0)
+    return out, _lse(M, L)

@@ -276,7 +276,51 @@ def check_backward_rows_partition(o):
         assert np.max(np.abs(dv_sum - dv)) < 1e-12
 
 
+def check_kvcache_is_the_last_rows_of_the_square_problem(o):
+    # Nq queries against Nk cached keys are the last Nq rows of the square
+    # problem whose queries fill all Nk positions (causal: query i at position
+    # Nk - Nq + i sees keys up to it), GQA included.
+    qf, k, v = _qkv(B=2, Hq=4, Hkv=2, N=17, d=5, seed=71)
+    for causal in (False, True):
+        fo, fl = o.attention_forward(qf, k, v, 0.6, causal)
+        for nq in (1, 3, 17):
+            ko, kl = o.attention_forward_kvcache(qf[:, :, 17 - nq:], k, v, 0.6, causal)
+            assert np.max(np.abs(ko - fo[:, :, 17 - nq:])) < 1e-13
+            assert np.max(np.abs(kl - fl[:, :, 17 - nq:])) < 1e-13
+
+
+def check_kvcache_single_query_sees_every_key(o):
+    # One new query is the last position: the causal mask hides nothing, and
+    # with a single cached key the output is that key's value (closed form).
+    q, k, v = _qkv(B=1, Hq=2, Hkv=1, N=9, d=4, seed=73)
+    q1 = q[:, :, -1:]
+    co, cl = o.attention_forward_kvcache(q1, k, v, 0.8, True)
+    no, nl = o.attention_forward_kvcache(q1, k, v, 0.8, False)
+    assert np.max(np.abs(co - no)) < 1e-15 and np.max(np.abs(cl - nl)) < 1e-15
+    so, sl = o.attention_forward_kvcache(q1, k[:, :, :1], v[:, :, :1], 0.8, True)
+    assert np.max(np.abs(so[0, :, 0] - v[0, 0, 0])) < 1e-15
+    assert np.max(np.abs(sl[0, :, 0] - 0.8 * q1[0, :, 0] @ k[0, 0, 0])) < 1e-14
+
+
+def check_merge_partial_states_matches_full(o):
+    # Softmax states of disjoint key chunks, merged with the rescale rule,
+    # give the softmax over all keys -- including chunks that are entirely
+    # masked for some rows under the causal mask.
+    q, k, v = _qkv(B=1, Hq=1, Hkv=1, N=29, d=6, seed=79)
+    for causal in (False, True):
+        fo, fl = o.attention_forward(q, k, v, 0.5, causal)
+        s = o.masked_scores(q[0, 0], k[0, 0], 0.5, causal)
+        cuts = [0, 4, 5, 17, 29]
+        states = [o.partial_state(s[:, a:b], v[0, 0, a:b]) for a, b in zip(cuts[:-1], cuts[1:])]
+        mo, ml = o.merge_partial_states(*(np.stack(x) for x in zip(*states)))
+        assert np.max(np.abs(mo - fo[0, 0])) < 1e-13
+        assert np.max(np.abs(ml - fl[0, 0])) < 1e-13
+
+
 ALL_CHECKS = [
+    check_kvcache_is_the_last_rows_of_the_square_problem,
+    check_kvcache_single_query_sees_every_key,
+    check_merge_partial_states_matches_full,
     check_backward_rows_partition,
     check_rows_sum_to_one,
     check_single_key_returns_value,
@@ -347,6 +391,27 @@ def _mut_kv_head(hq, Hq, Hkv):  # interleaved instead of contiguous groups
     return hq % Hkv
 
 
+def _mut_kvcache_top_left(q, k, v, scale, causal):  # queries placed at positions 0..Nq-1
+    q = np.asarray(q, float)
+    k = np.asarray(k, float)
+    v = np.asarray(v, float)
+    B, Hq, Nq, _ = q.shape
+    o = np.empty((B, Hq, Nq, v.shape[-1]))
+    lse = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            hk = ORACLE.kv_head_of(h, Hq, k.shape[1])
+            p, m, l = ORACLE.softmax_rows(ORACLE.masked_scores(q[b, h], k[b, hk], scale, causal))
+            o[b, h] = p @ v[b, hk]
+            lse[b, h] = m + np.log(l)
+    return o, lse
+
+
+def _mut_merge_no_rescale(ms, ls, os):  # sums added without the exp(m_s - M) factors
+    L = np.sum(ls, axis=0)
+    return np.sum(os, axis=0) / L[:, None], np.max(ms, axis=0) + np.log(L)
+
+
 ORIG = {name: getattr(ORACLE, name) for name in ("masked_scores", "softmax_rows", "score_gradient", "kv_head_of")}
 
 MUTATIONS = [
@@ -358,6 +423,8 @@ MUTATIONS = [
     ("softmax_rows", _mut_softmax_no_max),
     ("softmax_rows", _mut_softmax_wrong_norm),
     ("kv_head_of", _mut_kv_head),
+    ("attention_forward_kvcache", _mut_kvcache_top_left),
+    ("merge_partial_states", _mut_merge_no_rescale),
 ]
 
 
