@@ -451,6 +451,65 @@ def run_ours(args, rank, world, local):
 
 # --------------------------------------------------------- reference arm
 
+def run_kvcache(args, rank, world, local):
+    """Time fa_fwd_kvcache (decode over a KV cache) on one GPU: HBM throughput
+    of the bytes the method must move (K and V once, Q, O, LSE), against the
+    measured copy bandwidth."""
+    import torch
+
+    import exact_io_aware_61_b200 as fa
+
+    if world != 1:
+        raise SystemExit("--kvcache runs on one GPU")
+    B, Hq, Hkv, Nq, Nk, d = (int(x) for x in args.kvcache.split(","))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fa.load()
+    g = torch.Generator(device="cpu").manual_seed(SEED)
+    q = torch.randn((B, Hq, Nq, d), generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn((B, Hkv, Nk, d), generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn((B, Hkv, Nk, d), generator=g).to(torch.bfloat16).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(fa.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, Nq, Nk, d), 16), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = d ** -0.5
+    kv_bytes = 2 * B * Hkv * Nk * d * 2
+    flush = None if kv_bytes > 2 * 126e6 else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        fa.fa_fwd_kvcache(q, k, v, o, lse, ws, True, scale, stream)
+    torch.cuda.synchronize(dev)
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(physical_gpu_index(local))
+    sampler.start()
+    for e0, e1 in events:
+        if flush is not None:
+            flush.zero_()
+        e0.record(stream)
+        fa.fa_fwd_kvcache(q, k, v, o, lse, ws, True, scale, stream)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if fa.fa_last_device_status(stream) != fa.FA_OK:
+        raise RuntimeError("device status reports a timeout")
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in events)
+    nbytes = kv_bytes + 2 * B * Hq * Nq * d * 2 + 4 * B * Hq * Nq
+    peaks, src = load_peaks()
+    gbs = nbytes / ms / 1e6
+    print(json.dumps({
+        "metric": "KV-cache forward (decode) HBM throughput", "value": round(gbs, 1), "unit": "GB/s",
+        "higher_is_better": True, "ms": round(ms, 4), "steps": args.steps, "warmup": args.warmup,
+        "config": {"workload": f"causal bf16 KV-cache forward, B={B} Hq={Hq} Hkv={Hkv} Nq={Nq} Nk={Nk} d={d}",
+                   "l2": "no flush: K and V exceed twice the L2" if flush is None else
+                   "256 MB buffer written between timed launches"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes,
+                     "peak_note": f"{src} copy bandwidth"},
+        "tflops": round(4 * B * Hq * Nq * Nk * d / ms / 1e9, 2),
+        "clocks": clocks, "dtype": "bf16", "data": "synthetic: i.i.d. N(0,1) rounded to bf16, seeded"}))
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return  # rank 0 alone times the oracle; the others exit without work
@@ -498,6 +557,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fwd-only", action="store_true", help="skip the separate forward-only timed region")
+    ap.add_argument("--kvcache", default=None,
+                    help="B,Hq,Hkv,Nq,Nk,d: time the KV-cache (decode) forward instead of the benchmark step")
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d of a smaller case for profiling (default: the benchmark workload)")
     args = ap.parse_args(argv)
@@ -512,7 +573,9 @@ def main(argv=None):
     if world != args.gpus:
         if world == 1 and args.gpus > 1:
             ap.error(f"--gpus {args.gpus} needs a launch with torch.distributed.run (one rank per GPU)")
-    if args.impl == "reference":
+    if args.kvcache:
+        run_kvcache(args, rank, world, local)
+    elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
         run_ours(args, rank, world, local)

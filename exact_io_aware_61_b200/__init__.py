@@ -24,10 +24,13 @@ from ._lib import (  # noqa: F401
     fa_bwd_prep,
     fa_bwd_workspace_size,
     fa_fwd,
+    fa_fwd_kvcache,
+    fa_fwd_kvcache_workspace_size,
     fa_last_device_status,
     fa_selftest_wait_timeout,
     fa_set_wait_timeout_ns,
     forward,
+    forward_kvcache,
     load,
     status_string,
 )

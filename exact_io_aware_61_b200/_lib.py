@@ -28,6 +28,8 @@ EXPORTED = (
     "fa_bwd_dq",
     "fa_bwd_noalloc",
     "fa_bwd_workspace_size",
+    "fa_fwd_kvcache",
+    "fa_fwd_kvcache_workspace_size",
     "fa_status_string",
     "fa_last_device_status",
     "fa_set_wait_timeout_ns",
@@ -70,6 +72,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_bwd_noalloc.restype = i
         lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i]
         lib.fa_bwd_workspace_size.restype = sz
+        lib.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, f, i, i, vp]
+        lib.fa_fwd_kvcache.restype = i
+        lib.fa_fwd_kvcache_workspace_size.argtypes = [i, i, i, i, i, i]
+        lib.fa_fwd_kvcache_workspace_size.restype = sz
         lib.fa_status_string.argtypes = [i]
         lib.fa_status_string.restype = ctypes.c_char_p
         lib.fa_last_device_status.argtypes = [vp]
@@ -203,6 +209,36 @@ def fa_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, causal: bool, scale: float, 
                                _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd_noalloc")
+
+
+def fa_fwd_kvcache_workspace_size(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int) -> int:
+    return int(load().fa_fwd_kvcache_workspace_size(B, Hq, Hkv, Nq, Nk, d))
+
+
+def fa_fwd_kvcache(q, k, v, o, lse, workspace, causal: bool, scale: float, stream=None) -> None:
+    """Call ``fa_fwd_kvcache``: q [B,Hq,Nq,d] against k/v [B,Hkv,Nk,d] (Nk >= Nq); o like q, lse [B,Hq,Nq]."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse)):
+        _check_tensor(name, t, q.device)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    ws, nbytes = _ws(workspace)
+    rc = load().fa_fwd_kvcache(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ws, nbytes, B, Hq, Hkv, Nq, Nk, d,
+                               float(scale), int(bool(causal)), _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_kvcache")
+
+
+def forward_kvcache(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """Allocate O, LSE and the workspace with torch and run ``fa_fwd_kvcache``. Returns ``(o, lse)``."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    B, Hq, Nq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    nbytes = fa_fwd_kvcache_workspace_size(B, Hq, k.shape[1], Nq, k.shape[2], d)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    fa_fwd_kvcache(q, k, v, o, lse, ws, causal, scale, stream)
+    return o, lse
 
 
 def forward(q, k, v, causal: bool = False, scale: float | None = None, stream=None):

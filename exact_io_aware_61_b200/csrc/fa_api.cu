@@ -2,6 +2,7 @@
 // tensor maps, kernel selection and launches. One translation unit holds
 // every kernel so that they share the device status word.
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -22,6 +23,7 @@
 #include "fwd_f32.cuh"
 #include "bwd_sm100.cuh"
 #include "bwd2_sm100.cuh"
+#include "decode_sm100.cuh"
 
 namespace {
 
@@ -68,6 +70,16 @@ int check_device(int* dev_out) {
   return FA_OK;
 }
 
+// Dynamic shared memory of the KV-cache split kernels, one per row bucket.
+template <int HD, typename Set>
+void set_decode_attributes(Set& set) {
+  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 4>), fa::DecodeCfg<HD, 4>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 8>), fa::DecodeCfg<HD, 8>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 16>), fa::DecodeCfg<HD, 16>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 32>), fa::DecodeCfg<HD, 32>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 64>), fa::DecodeCfg<HD, 64>::SMEM_BYTES);
+}
+
 // Opt every kernel into its dynamic shared memory, once per device.
 int prepare_kernels(int dev) {
   static std::mutex mu;
@@ -85,6 +97,9 @@ int prepare_kernels(int dev) {
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<64>), fa::fwd_f32_smem_bytes<64>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<128>), fa::fwd_f32_smem_bytes<128>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<256>), fa::fwd_f32_smem_bytes<256>());
+  set_decode_attributes<64>(set);
+  set_decode_attributes<128>(set);
+  set_decode_attributes<256>(set);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64>), fa::Bwd2Cfg<64>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128>), fa::Bwd2Cfg<128>::SMEM_BYTES);
   if (e != cudaSuccess) return FA_ERR_CUDA;
@@ -384,6 +399,98 @@ int launch_bwd_dq(void* dq, void* ws, int B, int Hq, int Hkv, int N, int d, cuda
   return launch_convert(w.dq_acc, dq, static_cast<size_t>(B) * Hq * static_cast<size_t>(N) * d, stream);
 }
 
+// KV-cache forward: R query rows per KV head, S key splits of L keys (L a
+// multiple of 64). About two CTAs per SM of a 148-SM part, at least 256 keys
+// per split; a pure function of the sizes.
+struct DecodePlan {
+  int R, S, L;
+};
+
+DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk) {
+  DecodePlan dp;
+  dp.R = (Hq / Hkv) * Nq;
+  const long long pairs = static_cast<long long>(B) * Hkv;
+  const long long by_keys = std::max(1, (Nk + 255) / 256);
+  const long long by_sms = std::max(1LL, (296 + pairs - 1) / pairs);
+  const int s = static_cast<int>(std::min(by_keys, by_sms));
+  dp.L = ((Nk + s - 1) / s + 63) / 64 * 64;
+  dp.S = (Nk + dp.L - 1) / dp.L;
+  return dp;
+}
+
+// Validation of fa_fwd_kvcache's sizes: FA_OK, or the error to report.
+int check_kvcache_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < Nq || d < 1) return FA_ERR_INVALID;
+  if (Hq % Hkv != 0 || (causal != 0 && causal != 1) || !std::isfinite(scale)) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_INVALID;
+  if (static_cast<long long>(B) * Hq > INT32_MAX / 2 || Nk > INT32_MAX - 256) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 || (d != 64 && d != 128 && d != 256)) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(Hq / Hkv) * Nq > 64) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+size_t kvcache_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  const DecodePlan dp = decode_plan(B, Hq, Hkv, Nq, Nk);
+  return sizeof(float) * static_cast<size_t>(B) * Hkv * dp.S * dp.R * (static_cast<size_t>(d) + 2);
+}
+
+template <int HD, int RB>
+int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* ws, int B, int Hq,
+                  int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream) {
+  using C = fa::DecodeCfg<HD, RB>;
+  const DecodePlan dp = decode_plan(B, Hq, Hkv, Nq, Nk);
+  const uint64_t rows_kv = static_cast<uint64_t>(B) * Hkv;
+  CUtensorMap mk, mv;
+  int rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Nk, rows_kv, 64, C::BK);
+  if (rc == FA_OK) rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Nk, rows_kv, 64, C::BK);
+  if (rc != FA_OK) return rc;
+  float* part_o = static_cast<float*>(ws);
+  float* part_ml = part_o + rows_kv * dp.S * dp.R * HD;
+  fa::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.part_o = part_o;
+  p.part_ml = part_ml;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.R = dp.R;
+  p.S = dp.S;
+  p.L = dp.L;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.timeout_ns = timeout_now();
+  if (rows_kv > 65535) return FA_ERR_UNSUPPORTED;  // grid y
+  const dim3 grid(static_cast<unsigned>(dp.S), static_cast<unsigned>(rows_kv));
+  fa::fa_decode_split_kernel<HD, RB><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mk, mv, p);
+  if ((rc = launch_status(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, RB>))) != FA_OK) return rc;
+  fa::DecodeMergeParams mp;
+  mp.part_o = part_o;
+  mp.part_ml = part_ml;
+  mp.o = static_cast<__nv_bfloat16*>(o);
+  mp.lse = lse;
+  mp.Hq = Hq;
+  mp.Hkv = Hkv;
+  mp.Nq = Nq;
+  mp.R = dp.R;
+  mp.S = dp.S;
+  mp.rows = static_cast<int>(rows_kv * dp.R);
+  fa::fa_decode_merge_kernel<HD><<<static_cast<unsigned>((mp.rows + 7) / 8), 256, 0, stream>>>(mp);
+  return launch_status();
+}
+
+// Row bucket of the split kernel: the smallest of 4, 8, 16, 32, 64 that holds R.
+template <int HD>
+int launch_decode_rows(const void* q, const void* k, const void* v, void* o, float* lse, void* ws, int B, int Hq,
+                       int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream) {
+  const int R = (Hq / Hkv) * Nq;
+  if (R <= 4) return launch_decode<HD, 4>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
+  if (R <= 8) return launch_decode<HD, 8>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
+  if (R <= 16) return launch_decode<HD, 16>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
+  if (R <= 32) return launch_decode<HD, 32>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
+  return launch_decode<HD, 64>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
+}
+
 // Checks shared by the backward entry points. `ptrs` must all be 16-byte aligned and non-null.
 int check_bwd(std::initializer_list<const void*> ptrs, void* workspace, size_t workspace_bytes, int B, int Hq,
               int Hkv, int N, int d, float scale, int causal, int dtype, int* dev) {
@@ -567,6 +674,33 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
       return rc;
   }
   return launch_bwd_dq(dq, scratch, B, Hq, Hkv, N, d, s);
+}
+
+size_t fa_fwd_kvcache_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  if (check_kvcache_shape(B, Hq, Hkv, Nq, Nk, d, 1.0f, 0, FA_BF16) == FA_ERR_INVALID) return 0;
+  return kvcache_workspace_bytes(B, Hq, Hkv, Nq, Nk, d);
+}
+
+int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+                   size_t workspace_bytes, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   int dtype, fa_stream_t stream) {
+  int rc = check_kvcache_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (B == 0) return FA_OK;
+  for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(lse)})
+    if (!aligned16(ptr)) return FA_ERR_INVALID;
+  if (workspace == nullptr || workspace_bytes < kvcache_workspace_bytes(B, Hq, Hkv, Nq, Nk, d))
+    return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_INVALID;
+  int dev = 0;
+  if ((rc = check_device(&dev)) != FA_OK) return rc;
+  if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_decode_rows<64>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
+    case 128: return launch_decode_rows<128>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
+    default: return launch_decode_rows<256>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
+  }
 }
 
 int fa_last_device_status(fa_stream_t stream) {

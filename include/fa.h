@@ -194,6 +194,47 @@ FA_API int fa_bwd_noalloc(const void* q, const void* k, const void* v, const voi
                    int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                    int dtype, fa_stream_t stream);
 
+/*
+ * fa_fwd_kvcache_workspace_size -- bytes of device workspace fa_fwd_kvcache
+ * needs: per key split, the softmax state (max, sum, unnormalised output row)
+ * of each of the R = (Hq / Hkv) * Nq query rows of a KV head, float32:
+ * B * Hkv * S * R * (d + 2) * 4 bytes, S the number of key splits (a pure
+ * function of the sizes: S = min(ceil(Nk / 256), ceil(296 / (B * Hkv))), at
+ * least 1, then the keys are cut into S chunks of a multiple of 64). Returns
+ * 0 for invalid sizes.
+ */
+FA_API size_t fa_fwd_kvcache_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+
+/*
+ * fa_fwd_kvcache -- forward pass of Nq new queries against Nk >= Nq cached
+ * keys (decoding, or a short chunk of prefill, over a KV cache).
+ *
+ *   q [B][Hq][Nq][d], k, v [B][Hkv][Nk][d]   inputs (bf16)
+ *   o [B][Hq][Nq][d]                         output (bf16)
+ *   lse [B][Hq][Nq]                          output, float32, natural log of
+ *                                            the scaled scores
+ *   workspace, workspace_bytes               scratch owned by the caller,
+ *                                            >= fa_fwd_kvcache_workspace_size()
+ *                                            bytes, 16-byte aligned
+ *   scale, causal                            as for fa_fwd; query i is at key
+ *                                            position Nk - Nq + i, and with
+ *                                            causal = 1 it sees keys 0 .. Nk - Nq + i
+ * The pages name the KV cache as what now limits serving (fanfani.net
+ * "FlashAttention", "The backward pass, and where the memory saving comes
+ * from") and define the running-state rescale this uses to merge key splits
+ * ("A pinch of math: making the softmax work in pieces"). Two kernels run in
+ * stream order: one CTA per (batch, KV head, key split) computes each split's
+ * state for all R = (Hq / Hkv) * Nq query rows of the KV head (K and V are
+ * read from HBM once), then a merge kernel writes O and LSE. Supports dtype
+ * FA_BF16 with d in {64, 128, 256} and R <= 64; other cases return
+ * FA_ERR_UNSUPPORTED. Nq > Nk or Nq < 1 returns FA_ERR_INVALID; B == 0 is a
+ * no-op. On error nothing is written.
+ */
+FA_API int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* lse,
+                   void* workspace, size_t workspace_bytes,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   int dtype, fa_stream_t stream);
+
 /* Human-readable name of a fa_status value (static string, never NULL). */
 FA_API const char* fa_status_string(int status);
 

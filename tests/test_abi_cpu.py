@@ -114,6 +114,45 @@ def test_validation_before_any_device_work(lib):
     assert lib.fa_selftest_wait_timeout(0, None) == fa.FA_ERR_INVALID
 
 
+def _decode_plan(B, Hq, Hkv, Nq, Nk):
+    """Rows per KV head, key splits and keys per split of the KV-cache forward:
+    about 296 CTAs, at least 256 keys per split, splits a multiple of 64 keys."""
+    pairs = B * Hkv
+    s = min(max(1, (Nk + 255) // 256), max(1, -(-296 // pairs)))
+    L = (-(-Nk // s) + 63) // 64 * 64
+    return (Hq // Hkv) * Nq, -(-Nk // L), L
+
+
+def test_kvcache_workspace_formula(lib):
+    for shape in ((1, 32, 8, 1, 32768, 128), (8, 32, 8, 1, 32768, 128), (2, 8, 2, 4, 1000, 64),
+                  (1, 2, 1, 16, 16, 256), (64, 16, 16, 1, 4096, 128)):
+        B, Hq, Hkv, Nq, Nk, d = shape
+        R, S, L = _decode_plan(B, Hq, Hkv, Nq, Nk)
+        assert (S - 1) * L < Nk <= S * L and L % 64 == 0
+        assert fa.fa_fwd_kvcache_workspace_size(*shape) == 4 * B * Hkv * S * R * (d + 2), shape
+    assert fa.fa_fwd_kvcache_workspace_size(1, 2, 1, 9, 8, 64) == 0  # Nq > Nk
+    assert fa.fa_fwd_kvcache_workspace_size(1, 3, 2, 1, 64, 64) == 0  # Hq not a multiple of Hkv
+
+
+def test_kvcache_validation_before_any_device_work(lib):
+    def call(B=1, Hq=4, Hkv=2, Nq=1, Nk=100, d=128, scale=0.1, causal=1, dtype=0, ws_bytes=1 << 30):
+        p = ctypes.c_void_p(64)
+        return lib.fa_fwd_kvcache(p, p, p, p, p, p, ws_bytes, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, None)
+    assert call(Nq=101) == fa.FA_ERR_INVALID   # more queries than cached keys
+    assert call(Nq=0) == fa.FA_ERR_INVALID
+    assert call(Hq=3) == fa.FA_ERR_INVALID
+    assert call(causal=2) == fa.FA_ERR_INVALID
+    assert call(scale=float("nan")) == fa.FA_ERR_INVALID
+    assert call(dtype=1) == fa.FA_ERR_UNSUPPORTED  # fp32
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(Hq=32, Hkv=1, Nq=3) == fa.FA_ERR_UNSUPPORTED  # 96 query rows per KV head > 64
+    assert call(ws_bytes=16) == fa.FA_ERR_WORKSPACE
+    assert call(B=0) == fa.FA_OK  # empty problem
+    m = ctypes.c_void_p(66)
+    p = ctypes.c_void_p(64)
+    assert lib.fa_fwd_kvcache(p, m, p, p, p, p, 1 << 30, 1, 4, 2, 1, 100, 128, 0.1, 1, 0, None) == fa.FA_ERR_INVALID
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     from exact_io_aware_61_b200 import _lib
     saved = _lib._handle

@@ -233,6 +233,65 @@ def test_bwd_gqa_causal_b1_h32_kv8_n16384_d128(fa):
     assert torch.isfinite(dk.float()).all()
 
 
+# ------------------------------------------------------- KV-cache forward
+
+KVCACHE_SHAPES = [  # (B, Hq, Hkv, Nq, Nk, d)
+    (2, 8, 2, 1, 1000, 128),   # GQA decode, ragged Nk, several key splits
+    (1, 4, 4, 4, 777, 64),     # MHA, four new queries
+    (1, 32, 1, 2, 4096, 128),  # MQA, 64 query rows per KV head
+    (3, 8, 8, 1, 64, 256),     # one key tile
+    (1, 2, 1, 16, 16, 128),    # Nq = Nk: the square problem
+    (1, 16, 2, 8, 5000, 256),  # 64 rows per KV head at d = 256
+    (2, 4, 1, 1, 1, 64),       # a single cached key
+]
+
+
+def _kvcache_inputs(B, Hq, Hkv, Nq, Nk, d, seed):
+    # the new queries are the last Nq rows of a seeded square problem
+    inp = INP.make_inputs(B, Hq, Hkv, Nk, d, "bf16", seed=seed)
+    return inp["q"][:, :, Nk - Nq:].contiguous(), inp["k"], inp["v"]
+
+
+@pytest.mark.parametrize("shape", KVCACHE_SHAPES, ids=lambda s: "b%d_h%d_kv%d_nq%d_nk%d_d%d" % s)
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_kvcache_bf16(fa, shape, causal):
+    B, Hq, Hkv, Nq, Nk, d = shape
+    q, k, v = _kvcache_inputs(B, Hq, Hkv, Nq, Nk, d, seed=Nk + 7 * Nq + d)
+    o, lse = fa.forward_kvcache(_to_dev(q), _to_dev(k), _to_dev(v), causal=causal, scale=d ** -0.5)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.FA_OK
+    ro, rl = ORACLE.attention_forward_kvcache(INP.as_f64(q), INP.as_f64(k), INP.as_f64(v), d ** -0.5, causal)
+    assert np.max(np.abs(INP.as_f64(o) - ro)) <= O_TOL_BF16
+    assert np.max(np.abs(INP.as_f64(lse) - rl)) <= LSE_TOL_BF16
+
+
+def test_fwd_kvcache_decode_b8_h32_kv8_nk32768_d128(fa):
+    """One new token per sequence against a 32k-token cache, the whole batch
+    against the full oracle (one score row per head)."""
+    B, Hq, Hkv, Nq, Nk, d = 8, 32, 8, 1, 32768, 128
+    g = torch.Generator(device="cpu").manual_seed(32768)
+    q = torch.randn((B, Hq, Nq, d), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, Hkv, Nk, d), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Hkv, Nk, d), generator=g).to(torch.bfloat16)
+    o, lse = fa.forward_kvcache(_to_dev(q), _to_dev(k), _to_dev(v), causal=True, scale=d ** -0.5)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.FA_OK
+    ro, rl = ORACLE.attention_forward_kvcache(INP.as_f64(q), INP.as_f64(k), INP.as_f64(v), d ** -0.5, True)
+    assert np.max(np.abs(INP.as_f64(o) - ro)) <= O_TOL_BF16
+    assert np.max(np.abs(INP.as_f64(lse) - rl)) <= LSE_TOL_BF16
+
+
+def test_fwd_kvcache_square_case_matches_fwd(fa):
+    """With Nq = Nk the KV-cache path computes the square causal problem."""
+    inp = INP.make_inputs(1, 8, 2, 8, 128, "bf16", seed=88)
+    q, k, v = (_to_dev(inp[n]) for n in "qkv")
+    o1, l1 = fa.forward_kvcache(q, k, v, causal=True)
+    o2, l2 = fa.forward(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert float((o1.float() - o2.float()).abs().max()) <= O_TOL_BF16
+    assert float((l1 - l2).abs().max()) <= LSE_TOL_BF16
+
+
 # ---------------------------------------------------------- ABI behaviour
 
 def test_abi_rejects_bad_arguments_without_writing(fa):
