@@ -156,11 +156,11 @@ __global__ void __launch_bounds__(256, (DecodeCfg<HD, RB>::MIN_BLOCKS))
   const int cc = tid % C::CHUNKS;
   const int pr = KS > 1 ? (tid / C::CHUNKS) % RB : tid / C::CHUNKS;
   const int ks = KS > 1 ? tid / (C::CHUNKS * RB) : 0;
-  float acc[PROWS][8];
+  uint64_t acc[PROWS][4];  // packed f32 pairs: columns (2x, 2x + 1)
 #pragma unroll
   for (int k = 0; k < PROWS; ++k)
 #pragma unroll
-    for (int x = 0; x < 8; ++x) acc[k][x] = 0.f;
+    for (int x = 0; x < 4; ++x) acc[k][x] = 0ull;
 
   bool ok = true;
   for (int t = 0; t < n_tiles; ++t) {
@@ -169,23 +169,25 @@ __global__ void __launch_bounds__(256, (DecodeCfg<HD, RB>::MIN_BLOCKS))
     const uint32_t kt = sK + s * C::TILE_BYTES, vt = sV + s * C::TILE_BYTES;
     const int kg = k_begin + t * BK + key;  // this thread's key position
     if (ok) {
-      float dot[C::SROWS];
+      uint64_t dot2[C::SROWS];  // packed partial dot products (even, odd columns)
 #pragma unroll
-      for (int k = 0; k < C::SROWS; ++k) dot[k] = 0.f;
+      for (int k = 0; k < C::SROWS; ++k) dot2[k] = 0ull;
 #pragma unroll 4
       for (int c = 0; c < HD / 8; ++c) {
         uint4 w;
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
                      : "r"(swz_chunk<HD>(kt, key, c)));
-        float kf[8];
-        bf16x8_to_f32(w, kf);
+        const uint64_t k01 = pack2(bf16_lo(w.x), bf16_hi(w.x)), k23 = pack2(bf16_lo(w.y), bf16_hi(w.y));
+        const uint64_t k45 = pack2(bf16_lo(w.z), bf16_hi(w.z)), k67 = pack2(bf16_lo(w.w), bf16_hi(w.w));
 #pragma unroll
         for (int k = 0; k < C::SROWS; ++k) {
           const float4* qr = reinterpret_cast<const float4*>(sQ + (rg + 4 * k) * HD + 8 * c);
           const float4 qa = qr[0], qb = qr[1];
-          dot[k] = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3], dot[k]))));
-          dot[k] = fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], dot[k]))));
+          dot2[k] = ffma2(pack2(qa.x, qa.y), k01, dot2[k]);
+          dot2[k] = ffma2(pack2(qa.z, qa.w), k23, dot2[k]);
+          dot2[k] = ffma2(pack2(qb.x, qb.y), k45, dot2[k]);
+          dot2[k] = ffma2(pack2(qb.z, qb.w), k67, dot2[k]);
         }
       }
 #pragma unroll
@@ -193,7 +195,9 @@ __global__ void __launch_bounds__(256, (DecodeCfg<HD, RB>::MIN_BLOCKS))
         const int r = rg + 4 * k;
         const int pos = p.Nk - p.Nq + (r % p.Nq);
         const bool vis = r < R && kg < k_end && (!p.causal || kg <= pos);
-        sP[r * BK + key] = vis ? dot[k] * p.scale_log2 : -INFINITY;
+        float d0, d1;
+        unpack2(dot2[k], d0, d1);
+        sP[r * BK + key] = vis ? (d0 + d1) * p.scale_log2 : -INFINITY;
       }
     }
     __syncthreads();
@@ -228,8 +232,9 @@ __global__ void __launch_bounds__(256, (DecodeCfg<HD, RB>::MIN_BLOCKS))
 #pragma unroll
       for (int k = 0; k < PROWS; ++k) {
         const float a = sAlpha[pr + C::ROW_STRIDE * k * (PROWS > 1)];
+        const uint64_t a2 = pack2(a, a);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) acc[k][x] *= a;
+        for (int x = 0; x < 4; ++x) acc[k][x] = fmul2(acc[k][x], a2);
       }
 #pragma unroll 4
       for (int jj = 0; jj < BK / KS; ++jj) {
@@ -238,13 +243,14 @@ __global__ void __launch_bounds__(256, (DecodeCfg<HD, RB>::MIN_BLOCKS))
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
                      : "r"(swz_chunk<HD>(vt, j, cc)));
-        float vf[8];
-        bf16x8_to_f32(w, vf);
+        const uint64_t v2[4] = {pack2(bf16_lo(w.x), bf16_hi(w.x)), pack2(bf16_lo(w.y), bf16_hi(w.y)),
+                                pack2(bf16_lo(w.z), bf16_hi(w.z)), pack2(bf16_lo(w.w), bf16_hi(w.w))};
 #pragma unroll
         for (int k = 0; k < PROWS; ++k) {
           const float pj = sP[(pr + C::ROW_STRIDE * k * (PROWS > 1)) * BK + j];
+          const uint64_t p2 = pack2(pj, pj);
 #pragma unroll
-          for (int x = 0; x < 8; ++x) acc[k][x] = fmaf(pj, vf[x], acc[k][x]);
+          for (int x = 0; x < 4; ++x) acc[k][x] = ffma2(p2, v2[x], acc[k][x]);
         }
       }
     }
@@ -258,17 +264,17 @@ __global__ void __launch_bounds__(256, (DecodeCfg<HD, RB>::MIN_BLOCKS))
   if (KS > 1) {
     float* red = reinterpret_cast<float*>(gbase);  // the K/V stages are free now
     if (ks > 0) {
-      float4* dst = reinterpret_cast<float4*>(red + ((ks - 1) * RB * C::CHUNKS + pr * C::CHUNKS + cc) * 8);
-      dst[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-      dst[1] = make_float4(acc[0][4], acc[0][5], acc[0][6], acc[0][7]);
+      uint64_t* dst = reinterpret_cast<uint64_t*>(red + ((ks - 1) * RB * C::CHUNKS + pr * C::CHUNKS + cc) * 8);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) dst[x] = acc[0][x];
     }
     __syncthreads();
     if (ks == 0) {
       for (int q2 = 1; q2 < KS; ++q2) {
-        const float4* src = reinterpret_cast<const float4*>(red + ((q2 - 1) * RB * C::CHUNKS + pr * C::CHUNKS + cc) * 8);
-        const float4 a0 = src[0], a1 = src[1];
-        acc[0][0] += a0.x; acc[0][1] += a0.y; acc[0][2] += a0.z; acc[0][3] += a0.w;
-        acc[0][4] += a1.x; acc[0][5] += a1.y; acc[0][6] += a1.z; acc[0][7] += a1.w;
+        const uint64_t* src =
+            reinterpret_cast<const uint64_t*>(red + ((q2 - 1) * RB * C::CHUNKS + pr * C::CHUNKS + cc) * 8);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) acc[0][x] = fadd2(acc[0][x], src[x]);
       }
     }
   }
@@ -277,9 +283,9 @@ __global__ void __launch_bounds__(256, (DecodeCfg<HD, RB>::MIN_BLOCKS))
     for (int k = 0; k < PROWS; ++k) {
       const int r = pr + C::ROW_STRIDE * k * (PROWS > 1);
       if (r < R) {
-        float4* dst = reinterpret_cast<float4*>(p.part_o + (part * R + r) * HD + 8 * cc);
-        dst[0] = make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
-        dst[1] = make_float4(acc[k][4], acc[k][5], acc[k][6], acc[k][7]);
+        uint64_t* dst = reinterpret_cast<uint64_t*>(p.part_o + (part * R + r) * HD + 8 * cc);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) dst[x] = acc[k][x];
       }
     }
   }

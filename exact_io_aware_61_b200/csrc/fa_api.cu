@@ -400,7 +400,7 @@ int launch_bwd_dq(void* dq, void* ws, int B, int Hq, int Hkv, int N, int d, cuda
 }
 
 // KV-cache forward: R query rows per KV head, S key splits of L keys (L a
-// multiple of 64). About two CTAs per SM of a 148-SM part, at least 256 keys
+// multiple of 64). About four CTAs per SM of a 148-SM part, at least 256 keys
 // per split; a pure function of the sizes.
 struct DecodePlan {
   int R, S, L;
@@ -411,7 +411,7 @@ DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk) {
   dp.R = (Hq / Hkv) * Nq;
   const long long pairs = static_cast<long long>(B) * Hkv;
   const long long by_keys = std::max(1, (Nk + 255) / 256);
-  const long long by_sms = std::max(1LL, (296 + pairs - 1) / pairs);
+  const long long by_sms = std::max(1LL, (592 + pairs - 1) / pairs);
   const int s = static_cast<int>(std::min(by_keys, by_sms));
   dp.L = ((Nk + s - 1) / s + 63) / 64 * 64;
   dp.S = (Nk + dp.L - 1) / dp.L;

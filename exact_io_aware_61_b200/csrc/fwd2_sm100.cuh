@@ -65,34 +65,6 @@ FA_DEV float max3f(float a, float b, float c) {
   return d;
 }
 
-FA_DEV uint64_t pack2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-
-FA_DEV void unpack2(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-
-FA_DEV uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-
-FA_DEV uint64_t fadd2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-FA_DEV uint64_t fmul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
 // One 32-lane x 128-column TMEM load (one column per register), waited.
 FA_DEV void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
   asm volatile(

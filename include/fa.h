@@ -199,7 +199,7 @@ FA_API int fa_bwd_noalloc(const void* q, const void* k, const void* v, const voi
  * needs: per key split, the softmax state (max, sum, unnormalised output row)
  * of each of the R = (Hq / Hkv) * Nq query rows of a KV head, float32:
  * B * Hkv * S * R * (d + 2) * 4 bytes, S the number of key splits (a pure
- * function of the sizes: S = min(ceil(Nk / 256), ceil(296 / (B * Hkv))), at
+ * function of the sizes: S = min(ceil(Nk / 256), ceil(592 / (B * Hkv))), at
  * least 1, then the keys are cut into S chunks of a multiple of 64). Returns
  * 0 for invalid sizes.
  */

@@ -116,9 +116,9 @@ def test_validation_before_any_device_work(lib):
 
 def _decode_plan(B, Hq, Hkv, Nq, Nk):
     """Rows per KV head, key splits and keys per split of the KV-cache forward:
-    about 296 CTAs, at least 256 keys per split, splits a multiple of 64 keys."""
+    about 592 CTAs, at least 256 keys per split, splits a multiple of 64 keys."""
     pairs = B * Hkv
-    s = min(max(1, (Nk + 255) // 256), max(1, -(-296 // pairs)))
+    s = min(max(1, (Nk + 255) // 256), max(1, -(-592 // pairs)))
     L = (-(-Nk // s) + 63) // 64 * 64
     return (Hq // Hkv) * Nq, -(-Nk // L), L
 
