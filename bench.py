@@ -510,6 +510,59 @@ def run_kvcache(args, rank, world, local):
         "clocks": clocks, "dtype": "bf16", "data": "synthetic: i.i.d. N(0,1) rounded to bf16, seeded"}))
 
 
+def run_fwd_shape(args, rank, world, local):
+    """Time fa_fwd alone on one shape (B,Hq,Hkv,N,d,causal,dtype) on one GPU and
+    report TFLOP/s against the measured bf16 peak."""
+    import torch
+
+    import exact_io_aware_61_b200 as fa
+
+    if world != 1:
+        raise SystemExit("--fwd runs on one GPU")
+    B, Hq, Hkv, N, d, causal = (int(x) for x in args.fwd.split(",")[:6])
+    dtype = args.fwd.split(",")[6] if args.fwd.count(",") >= 6 else "bf16"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fa.load()
+    from exact_io_aware_61_b200 import inputs as inp_mod
+    host = inp_mod.make_inputs(B, Hq, Hkv, N, d, dtype, SEED)
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    flush = None if in_bytes > 2 * 126e6 else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        fa.fa_fwd(q, k, v, o, lse, causal, d ** -0.5, stream)
+    torch.cuda.synchronize(dev)
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(physical_gpu_index(local))
+    sampler.start()
+    for e0, e1 in events:
+        if flush is not None:
+            flush.zero_()
+        e0.record(stream)
+        fa.fa_fwd(q, k, v, o, lse, causal, d ** -0.5, stream)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if fa.fa_last_device_status(stream) != fa.FA_OK:
+        raise RuntimeError("device status reports a timeout")
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in events)
+    tflops = fwd_flops(B, Hq, N, d, bool(causal)) / ms / 1e9
+    peaks, src = load_peaks()
+    print(json.dumps({
+        "metric": "attention forward TFLOP/s", "value": round(tflops, 2), "unit": "TFLOP/s",
+        "higher_is_better": True, "ms": round(ms, 4), "steps": args.steps, "warmup": args.warmup,
+        "config": {"workload": f"{'causal' if causal else 'full'} {dtype} attention forward, "
+                               f"B={B} Hq={Hq} Hkv={Hkv} N={N} d={d}",
+                   "l2": "no flush: Q, K, V exceed twice the L2" if flush is None else
+                   "256 MB buffer written between timed launches"},
+        "pct_of_peak": round(100 * tflops / peaks["bf16_tflops"], 2), "peak_tflops": peaks["bf16_tflops"],
+        "peak_note": f"{src} bf16 GEMM (burst)", "clocks": clocks, "dtype": dtype,
+        "data": "synthetic: i.i.d. N(0,1), seeded"}))
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return  # rank 0 alone times the oracle; the others exit without work
@@ -557,6 +610,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fwd-only", action="store_true", help="skip the separate forward-only timed region")
+    ap.add_argument("--fwd", default=None,
+                    help="B,Hq,Hkv,N,d,causal[,dtype]: time the forward alone on that shape")
     ap.add_argument("--kvcache", default=None,
                     help="B,Hq,Hkv,Nq,Nk,d: time the KV-cache (decode) forward instead of the benchmark step")
     ap.add_argument("--shape", default=None,
@@ -575,6 +630,8 @@ def main(argv=None):
             ap.error(f"--gpus {args.gpus} needs a launch with torch.distributed.run (one rank per GPU)")
     if args.kvcache:
         run_kvcache(args, rank, world, local)
+    elif args.fwd:
+        run_fwd_shape(args, rank, world, local)
     elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
