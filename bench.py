@@ -45,7 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # of the dominant kernel, with the hash of the kernel source it was taken on.
 # Reported only while the source still hashes to the same value.
 TRAFFIC = {
-    # ncu --set full, benchmark shape, profiles/fa_bwd2_main_kernel_d128_causal_b2_h32_n8192.md
+    # dram__bytes_read.sum + dram__bytes_write.sum from one ncu --set full capture of
+    # one launch at the benchmark shape
     "bwd_main": {"src": "aec8e42337e23af8", "bytes": 824_382_208 + 501_768_448},
 }
 
