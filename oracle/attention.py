@@ -52,6 +52,12 @@ with the rescale rule of fanfani.net, section "A pinch of math: making the
 softmax work in pieces" (the same rule that carries the running state from one
 key block to the next).
 
+Variable-length batches (sequences of different lengths packed one after
+another, ``[tokens, heads, d]``, located by cumulative offsets) are attention
+within each sequence and nothing across sequences; the pages say nothing on
+layouts ("the softmax attention you asked for", synthetic.wiki, section "Where
+to be careful"), and the reading taken is the plain one.
+
 Layouts: Q, O, dO, dQ are ``[B, Hq, N, d]``; K, V, dK, dV are
 ``[B, Hkv, N, d]``; LSE and D are ``[B, Hq, N]``. All arithmetic is float64.
 """
@@ -72,6 +78,7 @@ __all__ = [
     "attention_backward_rows",
     "score_matrix_bytes",
     "attention_forward_kvcache",
+    "attention_forward_varlen",
     "partial_state",
     "merge_partial_states",
 ]
@@ -354,3 +361,37 @@ def merge_partial_states(ms, ls, os):
     with np.errstate(invalid="ignore", divide="ignore"):
         out = np.where(L[:, None] > 0, o / np.where(L > 0, L, 1.0)[:, None], 0.0)
     return out, _lse(M, L)
+
+
+def attention_forward_varlen(q, k, v, cu_q, cu_k, scale: float, causal: bool):
+    """Attention within each sequence of a packed variable-length batch.
+
+    ``q`` is ``[total_q, Hq, d]`` and ``k``, ``v`` are ``[total_k, Hkv, d]``:
+    sequence ``s`` owns query rows ``cu_q[s] .. cu_q[s+1]-1`` and key rows
+    ``cu_k[s] .. cu_k[s+1]-1`` (``cu_q``, ``cu_k`` non-decreasing, starting at
+    0, one entry more than sequences). A sequence may have fewer queries than
+    keys; its queries are then its last positions, as in
+    :func:`attention_forward_kvcache`. Returns ``(O [total_q, Hq, d], LSE
+    [total_q, Hq])``.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    cu_q = np.asarray(cu_q, dtype=np.int64)
+    cu_k = np.asarray(cu_k, dtype=np.int64)
+    if cu_q.shape != cu_k.shape or cu_q[0] != 0 or cu_k[0] != 0:
+        raise ValueError("cu_q and cu_k must start at 0 and have one entry per sequence boundary")
+    Hq, Hkv = q.shape[1], k.shape[1]
+    o = np.empty((q.shape[0], Hq, v.shape[-1]))
+    lse = np.empty((q.shape[0], Hq))
+    for s in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[s], cu_q[s + 1], cu_k[s], cu_k[s + 1]
+        if q1 - q0 > k1 - k0:
+            raise ValueError("a sequence has more queries than keys")
+        pos = (k1 - k0) - (q1 - q0) + np.arange(q1 - q0)
+        for h in range(Hq):
+            hk = kv_head_of(h, Hq, Hkv)
+            p, m, l = softmax_rows(masked_scores(q[q0:q1, h], k[k0:k1, hk], scale, causal, rows=pos))
+            o[q0:q1, h] = p @ v[k0:k1, hk]
+            lse[q0:q1, h] = _lse(m, l)
+    return o, lse

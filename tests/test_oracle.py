@@ -317,7 +317,51 @@ def check_merge_partial_states_matches_full(o):
         assert np.max(np.abs(ml - fl[0, 0])) < 1e-13
 
 
+def _varlen_pack(seed=83):
+    # three sequences: 5 queries / 9 keys, 7 / 7, 1 / 4; GQA 4 query heads on 2 KV heads
+    nq, nk = [5, 7, 1], [9, 7, 4]
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((sum(nq), 4, 3))
+    k = rng.standard_normal((sum(nk), 2, 3))
+    v = rng.standard_normal((sum(nk), 2, 3))
+    return q, k, v, np.cumsum([0] + nq), np.cumsum([0] + nk)
+
+
+def check_varlen_is_each_sequence_alone(o):
+    # A packed batch is each sequence's own (pinned) KV-cache problem: no key of
+    # another sequence reaches a query.
+    q, k, v, cq, ck = _varlen_pack()
+    for causal in (False, True):
+        po, pl = o.attention_forward_varlen(q, k, v, cq, ck, 0.7, causal)
+        for s in range(3):
+            qs = q[cq[s]:cq[s + 1]].transpose(1, 0, 2)[None]
+            ks = k[ck[s]:ck[s + 1]].transpose(1, 0, 2)[None]
+            vs = v[ck[s]:ck[s + 1]].transpose(1, 0, 2)[None]
+            so, sl = o.attention_forward_kvcache(qs, ks, vs, 0.7, causal)
+            assert np.max(np.abs(po[cq[s]:cq[s + 1]] - so[0].transpose(1, 0, 2))) < 1e-13
+            assert np.max(np.abs(pl[cq[s]:cq[s + 1]] - sl[0].T)) < 1e-13
+
+
+def check_varlen_sequence_order_invariance(o):
+    # Packing the same sequences in another order moves their rows and nothing else.
+    q, k, v, cq, ck = _varlen_pack(89)
+    order = [2, 0, 1]
+    qp = np.concatenate([q[cq[s]:cq[s + 1]] for s in order])
+    kp = np.concatenate([k[ck[s]:ck[s + 1]] for s in order])
+    vp = np.concatenate([v[ck[s]:ck[s + 1]] for s in order])
+    cqp = np.cumsum([0] + [cq[s + 1] - cq[s] for s in order])
+    ckp = np.cumsum([0] + [ck[s + 1] - ck[s] for s in order])
+    for causal in (False, True):
+        ao, al = o.attention_forward_varlen(q, k, v, cq, ck, 0.4, causal)
+        bo, bl = o.attention_forward_varlen(qp, kp, vp, cqp, ckp, 0.4, causal)
+        for i, s in enumerate(order):
+            assert np.max(np.abs(bo[cqp[i]:cqp[i + 1]] - ao[cq[s]:cq[s + 1]])) < 1e-14
+            assert np.max(np.abs(bl[cqp[i]:cqp[i + 1]] - al[cq[s]:cq[s + 1]])) < 1e-14
+
+
 ALL_CHECKS = [
+    check_varlen_is_each_sequence_alone,
+    check_varlen_sequence_order_invariance,
     check_kvcache_is_the_last_rows_of_the_square_problem,
     check_kvcache_single_query_sees_every_key,
     check_merge_partial_states_matches_full,
@@ -407,6 +451,14 @@ def _mut_kvcache_top_left(q, k, v, scale, causal):  # queries placed at position
     return o, lse
 
 
+def _mut_varlen_leak(q, k, v, cu_q, cu_k, scale, causal):  # every query sees the whole pack
+    kk = np.asarray(k, float)[None].transpose(0, 2, 1, 3)
+    vv = np.asarray(v, float)[None].transpose(0, 2, 1, 3)
+    qq = np.asarray(q, float)[None].transpose(0, 2, 1, 3)
+    o, lse = ORACLE.attention_forward_kvcache(qq, kk, vv, scale, False)
+    return o[0].transpose(1, 0, 2), lse[0].T
+
+
 def _mut_merge_no_rescale(ms, ls, os):  # sums added without the exp(m_s - M) factors
     L = np.sum(ls, axis=0)
     return np.sum(os, axis=0) / L[:, None], np.max(ms, axis=0) + np.log(L)
@@ -425,6 +477,7 @@ MUTATIONS = [
     ("kv_head_of", _mut_kv_head),
     ("attention_forward_kvcache", _mut_kvcache_top_left),
     ("merge_partial_states", _mut_merge_no_rescale),
+    ("attention_forward_varlen", _mut_varlen_leak),
 ]
 
 
