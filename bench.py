@@ -2,11 +2,11 @@
 """Throughput of exact causal attention, forward + backward, bf16, on B200.
 
 One step is the whole hot path over one batch: ``fa_fwd`` (O, LSE), then the
-three backward stages ``fa_bwd_prep`` (D, padded LSE, zeroed dQ accumulator),
-``fa_bwd_main`` (recompute, dK, dV, dQ accumulation) and ``fa_bwd_dq``
-(dQ to bf16), on B=2, Hq=Hkv=32, N=8192, d=128, causal, synthetic N(0,1)
-inputs rounded to bf16. FLOPs follow the usual convention: forward
-4*B*Hq*N^2*d, halved when causal; backward 2.5 times the forward.
+three backward stages ``fa_bwd_prep`` (D and the padded LSE), ``fa_bwd_dkdv``
+(key-side recompute: dK, dV) and ``fa_bwd_dq`` (query-side recompute: dQ),
+on B=2, Hq=Hkv=32, N=8192, d=128, causal, synthetic N(0,1) inputs rounded to
+bf16. FLOPs follow the usual convention: forward 4*B*Hq*N^2*d, halved when
+causal; backward 2.5 times the forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -41,14 +41,13 @@ SEED = 1003
 WORKLOAD_NAME = "causal bf16 attention forward+backward, B=2 Hq=32 Hkv=32 N=8192 d=128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# Measured DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
-# of the dominant kernel, with the hash of the kernel source it was taken on.
-# Reported only while the source still hashes to the same value.
-TRAFFIC = {
-    # dram__bytes_read.sum + dram__bytes_write.sum from one ncu --set full capture of
-    # one launch at the benchmark shape
-    "bwd_main": {"src": "aec8e42337e23af8", "bytes": 824_382_208 + 501_768_448},
-}
+SPEC_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor peak, vendor figure (context for pct_of_spec)
+
+# Counters of one ncu capture per kernel, with the hash of the kernel sources
+# they were taken on: DRAM bytes per launch (dram__bytes_read.sum +
+# dram__bytes_write.sum) and sm__pipe_tensor_cycles_active (% of peak). They
+# are reported only while the sources still hash to the same value.
+PROFILED = {}
 
 
 def fwd_flops(B, Hq, N, d, causal):
@@ -60,16 +59,29 @@ def bwd_flops(B, Hq, N, d, causal):
     return 2.5 * fwd_flops(B, Hq, N, d, causal)
 
 
+def kernel_flops(B, Hq, N, d, causal):
+    """Algorithmic FLOPs credited to each kernel, and the FLOPs it executes.
+
+    Each of the backward's five products (S, dP, dV, dK, dQ) costs half the
+    forward. The dK/dV kernel computes S^T, dP^T, dV and dK: four products,
+    all of them the method's own work. The dQ kernel computes S, dP and dQ;
+    only dQ is new work, S and dP are computed a second time so that dQ can be
+    accumulated on chip. The credited FLOPs add up to the convention's 2.5x.
+    """
+    f = fwd_flops(B, Hq, N, d, causal)
+    return {"fwd": (f, f), "bwd_dkdv": (2.0 * f, 2.0 * f), "bwd_dq": (0.5 * f, 1.5 * f)}
+
+
 def algorithmic_bytes(B, Hq, Hkv, N, d):
-    """Bytes each kernel must move at least once (bf16 tensors, f32 LSE/D/accumulator)."""
+    """Bytes each kernel must move at least once (bf16 tensors, f32 LSE/D)."""
     q = B * Hq * N * d * 2
     kv = B * Hkv * N * d * 2
     rows = B * Hq * N * 4
     return {
         "fwd": q + 2 * kv + q + rows,                     # read Q, K, V; write O, LSE
-        "bwd_prep": 2 * q + rows + 2 * rows + 2 * q,      # read O, dO, LSE; write D, LSE2, zero dQacc (f32)
-        "bwd_main": 2 * q + 2 * kv + 2 * rows + 2 * kv + 2 * q * 2,  # read Q,dO,K,V,LSE2,D; write dK,dV; dQacc add
-        "bwd_dq": 2 * q + q,                              # read dQacc (f32), write dQ
+        "bwd_prep": 2 * q + rows + 2 * rows,              # read O, dO, LSE; write D, LSE2
+        "bwd_dkdv": 2 * q + 2 * kv + 2 * rows + 2 * kv,   # read Q, dO, K, V, LSE2, D; write dK, dV
+        "bwd_dq": 2 * q + 2 * kv + 2 * rows + q,          # read Q, dO, K, V, LSE2, D; write dQ
     }
 
 
@@ -284,10 +296,10 @@ def run_ours(args, rank, world, local):
         fa.fa_bwd_prep(o, lse, do, ws, Hkv, stream)
         if ev is not None:
             ev[2].record(stream)
-        fa.fa_bwd_main(q, k, v, do, dk, dv, ws, CAUSAL, scale, stream)
+        fa.fa_bwd_dkdv(q, k, v, do, dk, dv, ws, CAUSAL, scale, stream)
         if ev is not None:
             ev[3].record(stream)
-        fa.fa_bwd_dq(dq, ws, Hkv, stream)
+        fa.fa_bwd_dq(q, k, v, do, dq, ws, CAUSAL, scale, stream)
         if ev is not None:
             ev[4].record(stream)
 
@@ -317,14 +329,14 @@ def run_ours(args, rank, world, local):
 
     elapsed_ms = start.elapsed_time(end)
     per_kernel = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in events)
-                  for i, name in enumerate(("fwd", "bwd_prep", "bwd_main", "bwd_dq"))}
+                  for i, name in enumerate(("fwd", "bwd_prep", "bwd_dkdv", "bwd_dq"))}
     max_ms = max_over_ranks(elapsed_ms, world, dev)
 
     f_fwd = fwd_flops(B, Hq, N, d, CAUSAL)
     f_bwd = bwd_flops(B, Hq, N, d, CAUSAL)
     step_flops = f_fwd + f_bwd
     value = world * step_flops * args.steps / (max_ms / 1e3) / 1e12
-    bwd_ms = per_kernel["bwd_prep"] + per_kernel["bwd_main"] + per_kernel["bwd_dq"]
+    bwd_ms = per_kernel["bwd_prep"] + per_kernel["bwd_dkdv"] + per_kernel["bwd_dq"]
 
     # forward alone: its own timed region (no backward kernels in between)
     fwd_only = None
@@ -378,8 +390,8 @@ def run_ours(args, rank, world, local):
             comp.wait_event(downloaded[s])  # step i-2's outputs have left this set
             fa.fa_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"], CAUSAL, scale, comp)
             fa.fa_bwd_prep(b["o"], b["lse"], b["do"], b["ws"], Hkv, comp)
-            fa.fa_bwd_main(b["q"], b["k"], b["v"], b["do"], b["dk"], b["dv"], b["ws"], CAUSAL, scale, comp)
-            fa.fa_bwd_dq(b["dq"], b["ws"], Hkv, comp)
+            fa.fa_bwd_dkdv(b["q"], b["k"], b["v"], b["do"], b["dk"], b["dv"], b["ws"], CAUSAL, scale, comp)
+            fa.fa_bwd_dq(b["q"], b["k"], b["v"], b["do"], b["dq"], b["ws"], CAUSAL, scale, comp)
             computed[s].record(comp)
             down.wait_event(computed[s])
             with torch.cuda.stream(down):
@@ -425,20 +437,30 @@ def run_ours(args, rank, world, local):
     peak_tf = float(peaks["bf16_tflops"])
     hbm = float(peaks["hbm_gbs"])
     nbytes = algorithmic_bytes(B, Hq, Hkv, N, d)
-    kernels = {
-        "fwd": {"ms": per_kernel["fwd"], "tflops": f_fwd / per_kernel["fwd"] / 1e9,
-                "gbs": nbytes["fwd"] / per_kernel["fwd"] / 1e6},
-        "bwd_main": {"ms": per_kernel["bwd_main"], "tflops": f_bwd / per_kernel["bwd_main"] / 1e9,
-                     "gbs": nbytes["bwd_main"] / per_kernel["bwd_main"] / 1e6},
-        "bwd_prep": {"ms": per_kernel["bwd_prep"], "gbs": nbytes["bwd_prep"] / per_kernel["bwd_prep"] / 1e6},
-        "bwd_dq": {"ms": per_kernel["bwd_dq"], "gbs": nbytes["bwd_dq"] / per_kernel["bwd_dq"] / 1e6},
-    }
-    dominant = "bwd_main" if per_kernel["bwd_main"] >= per_kernel["fwd"] else "fwd"
-    dom_flops = f_bwd if dominant == "bwd_main" else f_fwd
-    achieved = dom_flops / per_kernel[dominant] / 1e9
+    kf = kernel_flops(B, Hq, N, d, CAUSAL)
     src_hash = kernel_source_hash()
-    traffic = TRAFFIC.get(dominant)
-    traffic_val = traffic["bytes"] if traffic and traffic.get("src") == src_hash else None
+    names = {"fwd": f"fa_fwd_bf16_2tile_kernel<{d}>", "bwd_prep": f"fa_bwd_prep_kernel<{d}>",
+             "bwd_dkdv": f"fa_bwd_dkdv_kernel<{d}>", "bwd_dq": f"fa_bwd_dq_kernel<{d}>"}
+    kernels = {}
+    for name, ms in per_kernel.items():
+        e = {"kernel": names[name], "ms": round(ms, 4), "gbs": round(nbytes[name] / ms / 1e6, 1)}
+        if name in kf:
+            credited, executed = kf[name]
+            e["tflops"] = round(credited / ms / 1e9, 2)
+            e["executed_tflops"] = round(executed / ms / 1e9, 2)
+            e["pct_of_peak"] = round(100 * credited / ms / 1e9 / peak_tf, 2)
+        prof = PROFILED.get(name)
+        if prof and prof.get("src") == src_hash:
+            e["tensor_pipe_active_pct"] = prof.get("tensor_pipe_active_pct")
+            e["dram_bytes"] = prof.get("dram_bytes")
+        kernels[name] = e
+    dominant = max(kf, key=lambda n: per_kernel[n])
+    credited, executed = kf[dominant]
+    achieved = credited / per_kernel[dominant] / 1e9
+    prof = PROFILED.get(dominant)
+    fresh = bool(prof) and prof.get("src") == src_hash
+    traffic_val = prof.get("dram_bytes") if fresh else None
+    tensor_active = prof.get("tensor_pipe_active_pct") if fresh else None
 
     out = {
         "metric": METRIC,
@@ -462,10 +484,19 @@ def run_ours(args, rank, world, local):
                         "bwd": round(100 * f_bwd / bwd_ms / 1e9 / peak_tf, 2),
                         "step": round(100 * value / world / peak_tf, 2),
                         "peak_tflops": peak_tf, "peak_source": f"{peak_src} bf16_tflops (burst)"},
-        "kernels": {k: {kk: round(vv, 4) for kk, vv in v.items()} for k, v in kernels.items()},
-        "roofline": {"kernel": f"fa_bwd2_main_kernel<{d}>" if dominant == "bwd_main" else f"fa_fwd_bf16_2tile_kernel<{d}>",
-                     "bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak_tf, 4), "traffic": traffic_val,
+        "pct_of_spec": {"fwd": round(100 * f_fwd / per_kernel["fwd"] / 1e9 / SPEC_BF16_TFLOPS, 2),
+                        "bwd": round(100 * f_bwd / bwd_ms / 1e9 / SPEC_BF16_TFLOPS, 2),
+                        "step": round(100 * value / world / SPEC_BF16_TFLOPS, 2),
+                        "spec_tflops": SPEC_BF16_TFLOPS,
+                        "spec_source": "vendor dense bf16 figure (the 2:4-sparse figure halved)"},
+        "hbm_gbs": {"fwd": kernels["fwd"]["gbs"],
+                    "bwd": round(sum(nbytes[n] for n in ("bwd_prep", "bwd_dkdv", "bwd_dq")) / bwd_ms / 1e6, 1),
+                    "peak_gbs": hbm},
+        "kernels": kernels,
+        "roofline": {"kernel": names[dominant], "bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4), "traffic": traffic_val,
+                     "tensor_pipe_active": tensor_active,
+                     "algorithmic_flops": credited, "executed_flops": executed,
                      "algorithmic_bytes": nbytes[dominant],
                      "peak_note": f"{peak_src} (burst bf16 GEMM)", "hbm_peak_gbs": hbm},
         "gpu_launches": 4 * args.steps,

@@ -19,8 +19,9 @@ from ._lib import (  # noqa: F401
     FAError,
     backward,
     fa_bwd,
+    fa_bwd_dkdv,
     fa_bwd_dq,
-    fa_bwd_main,
+    fa_bwd_noalloc,
     fa_bwd_prep,
     fa_bwd_workspace_size,
     fa_fwd,

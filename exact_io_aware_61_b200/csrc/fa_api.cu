@@ -22,7 +22,8 @@
 #include "fwd2_sm100.cuh"
 #include "fwd_f32.cuh"
 #include "bwd_sm100.cuh"
-#include "bwd2_sm100.cuh"
+#include "bwd_dkdv_sm100.cuh"
+#include "bwd_dq_sm100.cuh"
 #include "decode_sm100.cuh"
 
 namespace {
@@ -100,8 +101,10 @@ int prepare_kernels(int dev) {
   set_decode_attributes<64>(set);
   set_decode_attributes<128>(set);
   set_decode_attributes<256>(set);
-  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64>), fa::Bwd2Cfg<64>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128>), fa::Bwd2Cfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd_dkdv_kernel<64>), fa::BwdKVCfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd_dkdv_kernel<128>), fa::BwdKVCfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd_dq_kernel<64>), fa::BwdQCfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd_dq_kernel<128>), fa::BwdQCfg<128>::SMEM_BYTES);
   if (e != cudaSuccess) return FA_ERR_CUDA;
   done[dev] = true;
   return FA_OK;
@@ -260,9 +263,9 @@ int launch_fwd_f32(const void* q, const void* k, const void* v, void* o, float* 
 size_t padded_rows(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 
 // How many CTAs share the query heads of one (KV head, 128-key tile) in the
-// backward: 1 unless B * Hkv * (key tiles) is below 592 (4 CTAs per SM of a
-// 148-SM part), then the smallest divisor of the group size that reaches it,
-// or the group size. A pure function of the shape, so the workspace size
+// dK/dV kernel: 1 unless B * Hkv * (key tiles) is below 592 (4 CTAs per SM of
+// a 148-SM part), then the smallest divisor of the group size that reaches
+// it, or the group size. A pure function of the shape, so the workspace size
 // does not depend on the device.
 int bwd_head_split(int B, int Hq, int Hkv, int N) {
   const long long ctas = static_cast<long long>(B) * Hkv * static_cast<long long>(padded_rows(N) / 128);
@@ -272,16 +275,21 @@ int bwd_head_split(int B, int Hq, int Hkv, int N) {
   return g;
 }
 
-// Workspace carve-up, all f32: D [B*Hq][Npad], LSE*log2(e) [B*Hq][Npad],
-// dQ accumulator [B*Hq][N][d]; when the backward splits a group's heads over
-// CTAs, also dK and dV accumulators [B*Hkv][N][d].
+// Workspace carve-up, all f32: D [B*Hq][Npad], LSE*log2(e) [B*Hq][Npad];
+// when the dK/dV kernel splits a group's heads over CTAs, also dK and dV
+// accumulators [B*Hkv][N][d].
 struct BwdWorkspace {
   float* delta;
   float* lse2;
-  float* dq_acc;
   float* dk_acc;  // null without a split
   float* dv_acc;
 };
+
+size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
+  const size_t rows_q = static_cast<size_t>(B) * Hq;
+  const size_t kv_acc = bwd_head_split(B, Hq, Hkv, N) > 1 ? 2 * static_cast<size_t>(B) * Hkv * N * d : 0;
+  return sizeof(float) * (2 * rows_q * padded_rows(N) + kv_acc);
+}
 
 BwdWorkspace carve(void* ws, int B, int Hq, int Hkv, int N, int d) {
   const size_t npad = padded_rows(N);
@@ -290,113 +298,160 @@ BwdWorkspace carve(void* ws, int B, int Hq, int Hkv, int N, int d) {
   BwdWorkspace w;
   w.delta = static_cast<float*>(ws);
   w.lse2 = w.delta + rows_q * npad;
-  w.dq_acc = w.lse2 + rows_q * npad;
   const bool split = bwd_head_split(B, Hq, Hkv, N) > 1;
-  w.dk_acc = split ? w.dq_acc + rows_q * static_cast<size_t>(N) * d : nullptr;
+  w.dk_acc = split ? w.lse2 + rows_q * npad : nullptr;
   w.dv_acc = split ? w.dk_acc + kv_elems : nullptr;
   return w;
 }
 
-// f32 -> bf16 rounding of n elements (a multiple of 4) on `stream`.
-int launch_convert(const float* acc, void* out, size_t n, cudaStream_t stream) {
-  const size_t n4 = n / 4;
+unsigned grid_stride_blocks(size_t n4) {
   const size_t want = (n4 + 255) / 256;
-  const unsigned grid = static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
-  fa::fa_bwd_dq_kernel<<<grid, 256, 0, stream>>>(acc, static_cast<__nv_bfloat16*>(out), n4);
-  return launch_status();
+  return static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
 }
 
-int launch_zero(float* p, size_t n, cudaStream_t stream) {
-  const size_t n4 = n / 4;
-  const size_t want = (n4 + 255) / 256;
-  const unsigned grid = static_cast<unsigned>(want < 148 * 16 ? want : 148 * 16);
-  fa::fa_zero_f32_kernel<<<grid, 256, 0, stream>>>(p, n4);
-  return launch_status();
-}
-
-template <int HD>
-int launch_bwd_prep(const void* o, const float* lse, const void* dO, void* ws, int B, int Hq, int Hkv, int N,
-                    cudaStream_t stream) {
-  const BwdWorkspace w = carve(ws, B, Hq, Hkv, N, HD);
-  const size_t npad = padded_rows(N);
+// Everything the backward's launches need, built (tensor maps encoded, grid
+// sizes checked) before the first of them is queued, so that every error
+// return of a backward entry point comes before any kernel runs.
+struct BwdPlan {
+  int d;
+  cudaStream_t stream;
+  BwdWorkspace w;
+  size_t kv_elems;
+  int split;
+  // prep
   fa::BwdPrepParams pp;
-  pp.o = static_cast<const __nv_bfloat16*>(o);
-  pp.dO = static_cast<const __nv_bfloat16*>(dO);
-  pp.lse = lse;
-  pp.ws_delta = w.delta;
-  pp.ws_lse2 = w.lse2;
-  pp.dq_acc = w.dq_acc;
-  pp.N = N;
-  pp.Npad = static_cast<int>(npad);
-  const long long blocks = static_cast<long long>(npad / 32) * B * Hq;
-  if (blocks > INT32_MAX) return FA_ERR_INVALID;
-  fa::fa_bwd_prep_kernel<HD><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(pp);
-  return launch_status();
-}
+  unsigned prep_blocks;
+  // dK/dV
+  CUtensorMap kv_mq, kv_mdo;
+  fa::BwdKVParams kp;
+  unsigned kv_blocks;
+  // dQ
+  CUtensorMap q_mk, q_mv;
+  fa::BwdQParams qp;
+  unsigned q_blocks;
+};
 
-template <int HD>
-int launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* ws,
-                    int B, int Hq, int Hkv, int N, float scale, int causal, cudaStream_t stream) {
-  using C = fa::Bwd2Cfg<HD>;
-  const BwdWorkspace w = carve(ws, B, Hq, Hkv, N, HD);
-  const int split = bwd_head_split(B, Hq, Hkv, N);
-  const size_t kv_elems = static_cast<size_t>(B) * Hkv * static_cast<size_t>(N) * HD;
+// stages: bit 0 prep, bit 1 dK/dV, bit 2 dQ. Pointers a stage does not use may be null.
+int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const void* v, const void* o,
+             const float* lse, const void* dO, void* dq, void* dk, void* dv, void* ws, int B, int Hq, int Hkv,
+             int N, int d, float scale, int causal, cudaStream_t stream) {
+  pl->d = d;
+  pl->stream = stream;
+  pl->w = carve(ws, B, Hq, Hkv, N, d);
+  pl->kv_elems = static_cast<size_t>(B) * Hkv * static_cast<size_t>(N) * d;
+  pl->split = bwd_head_split(B, Hq, Hkv, N);
   const size_t npad = padded_rows(N);
   const uint64_t rows_q = static_cast<uint64_t>(B) * Hq, rows_kv = static_cast<uint64_t>(B) * Hkv;
-  CUtensorMap mq, mk, mv, mdo, mdq;
-  int rc = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
-  if (rc == FA_OK) rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
-  if (rc == FA_OK) rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
-  if (rc == FA_OK) rc = make_map(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
-  if (rc == FA_OK) rc = make_map(&mdq, w.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, N, rows_q, 32, 128);
-  if (rc != FA_OK) return rc;
-  fa::Bwd2Params p;
-  p.ws_delta = w.delta;
-  p.ws_lse2 = w.lse2;
-  p.dq_acc = w.dq_acc;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.dk_acc = w.dk_acc;
-  p.dv_acc = w.dv_acc;
-  p.head_split = split;
-  p.BHkv = B * Hkv;
-  p.N = N;
-  p.Npad = static_cast<int>(npad);
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.num_tiles = static_cast<int>(npad / 128);
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.scale = scale;
-  p.causal = causal;
-  p.timeout_ns = timeout_now();
-  const long long blocks = static_cast<long long>(p.num_tiles) * B * Hkv * split;
-  if (blocks > INT32_MAX) return FA_ERR_INVALID;
-  // The kernel redistributes registers between warpgroups (setmaxnreg) on
-  // the assumption of exactly LAUNCH_REGS per thread at launch.
-  cudaFuncAttributes attr;
-  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>)) != cudaSuccess)
-    return FA_ERR_CUDA;
-  if (attr.numRegs != C::LAUNCH_REGS) {
-    if (verbose()) std::fprintf(stderr, "fa: backward built with %d registers, expected %d\n", attr.numRegs,
-                                C::LAUNCH_REGS);
-    return FA_ERR_UNSUPPORTED;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  const unsigned long long tmo = timeout_now();
+  if (stages & 1u) {
+    fa::BwdPrepParams& pp = pl->pp;
+    pp.o = static_cast<const __nv_bfloat16*>(o);
+    pp.dO = static_cast<const __nv_bfloat16*>(dO);
+    pp.lse = lse;
+    pp.ws_delta = pl->w.delta;
+    pp.ws_lse2 = pl->w.lse2;
+    pp.N = N;
+    pp.Npad = static_cast<int>(npad);
+    const long long blocks = static_cast<long long>(npad / 32) * B * Hq;
+    if (blocks > INT32_MAX) return FA_ERR_INVALID;
+    pl->prep_blocks = static_cast<unsigned>(blocks);
   }
-  if (split > 1) {
-    if ((rc = launch_zero(w.dk_acc, 2 * kv_elems, stream)) != FA_OK) return rc;  // dK and dV accumulators
+  if (stages & 2u) {
+    int rc = make_map(&pl->kv_mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, rows_q, 64, 64);
+    if (rc == FA_OK) rc = make_map(&pl->kv_mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, rows_q, 64, 64);
+    if (rc != FA_OK) return rc;
+    fa::BwdKVParams& kp = pl->kp;
+    kp.k = static_cast<const __nv_bfloat16*>(k);
+    kp.v = static_cast<const __nv_bfloat16*>(v);
+    kp.ws_delta = pl->w.delta;
+    kp.ws_lse2 = pl->w.lse2;
+    kp.dk = static_cast<__nv_bfloat16*>(dk);
+    kp.dv = static_cast<__nv_bfloat16*>(dv);
+    kp.dk_acc = pl->w.dk_acc;
+    kp.dv_acc = pl->w.dv_acc;
+    kp.head_split = pl->split;
+    kp.BHkv = B * Hkv;
+    kp.N = N;
+    kp.Npad = static_cast<int>(npad);
+    kp.Hq = Hq;
+    kp.Hkv = Hkv;
+    kp.num_tiles = static_cast<int>(npad / 128);
+    kp.scale_log2 = scale_log2;
+    kp.scale = scale;
+    kp.causal = causal;
+    kp.timeout_ns = tmo;
+    const long long blocks = static_cast<long long>(kp.num_tiles) * B * Hkv * pl->split;
+    if (blocks > INT32_MAX) return FA_ERR_INVALID;
+    pl->kv_blocks = static_cast<unsigned>(blocks);
   }
-  fa::fa_bwd2_main_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
-                                                                                                     mdq, p);
-  if ((rc = launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>))) != FA_OK) return rc;
-  if (split > 1) {
-    if ((rc = launch_convert(w.dk_acc, dk, kv_elems, stream)) != FA_OK) return rc;
-    if ((rc = launch_convert(w.dv_acc, dv, kv_elems, stream)) != FA_OK) return rc;
+  if (stages & 4u) {
+    int rc = make_map(&pl->q_mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, rows_kv, 64, 64);
+    if (rc == FA_OK) rc = make_map(&pl->q_mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, rows_kv, 64, 64);
+    if (rc != FA_OK) return rc;
+    fa::BwdQParams& qp = pl->qp;
+    qp.q = static_cast<const __nv_bfloat16*>(q);
+    qp.dO = static_cast<const __nv_bfloat16*>(dO);
+    qp.ws_delta = pl->w.delta;
+    qp.ws_lse2 = pl->w.lse2;
+    qp.dq = static_cast<__nv_bfloat16*>(dq);
+    qp.N = N;
+    qp.Npad = static_cast<int>(npad);
+    qp.Hq = Hq;
+    qp.Hkv = Hkv;
+    qp.BH = B * Hq;
+    qp.num_tiles = static_cast<int>(npad / 128);
+    qp.scale_log2 = scale_log2;
+    qp.scale = scale;
+    qp.causal = causal;
+    qp.timeout_ns = tmo;
+    const long long blocks = static_cast<long long>(qp.num_tiles) * B * Hq;
+    if (blocks > INT32_MAX) return FA_ERR_INVALID;
+    pl->q_blocks = static_cast<unsigned>(blocks);
   }
   return FA_OK;
 }
 
-int launch_bwd_dq(void* dq, void* ws, int B, int Hq, int Hkv, int N, int d, cudaStream_t stream) {
-  const BwdWorkspace w = carve(ws, B, Hq, Hkv, N, d);
-  return launch_convert(w.dq_acc, dq, static_cast<size_t>(B) * Hq * static_cast<size_t>(N) * d, stream);
+template <int HD>
+int launch_bwd_prep(const BwdPlan& pl) {
+  fa::fa_bwd_prep_kernel<HD><<<pl.prep_blocks, 256, 0, pl.stream>>>(pl.pp);
+  return launch_status();
+}
+
+template <int HD>
+int launch_bwd_dkdv(const BwdPlan& pl) {
+  using C = fa::BwdKVCfg<HD>;
+  if (pl.split > 1) {  // zero the f32 dK and dV accumulators (contiguous)
+    fa::fa_zero_f32_kernel<<<grid_stride_blocks(pl.kv_elems / 2), 256, 0, pl.stream>>>(pl.w.dk_acc,
+                                                                                      pl.kv_elems / 2);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  fa::fa_bwd_dkdv_kernel<HD><<<pl.kv_blocks, C::THREADS, C::SMEM_BYTES, pl.stream>>>(pl.kv_mq, pl.kv_mdo, pl.kp);
+  if (launch_status(reinterpret_cast<const void*>(&fa::fa_bwd_dkdv_kernel<HD>)) != FA_OK) return FA_ERR_CUDA;
+  if (pl.split > 1) {
+    const size_t n4 = pl.kv_elems / 4;
+    fa::fa_f32_to_bf16_kernel<<<grid_stride_blocks(n4), 256, 0, pl.stream>>>(pl.w.dk_acc, pl.kp.dk, n4);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+    fa::fa_f32_to_bf16_kernel<<<grid_stride_blocks(n4), 256, 0, pl.stream>>>(pl.w.dv_acc, pl.kp.dv, n4);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+template <int HD>
+int launch_bwd_dq(const BwdPlan& pl) {
+  using C = fa::BwdQCfg<HD>;
+  fa::fa_bwd_dq_kernel<HD><<<pl.q_blocks, C::THREADS, C::SMEM_BYTES, pl.stream>>>(pl.q_mk, pl.q_mv, pl.qp);
+  return launch_status(reinterpret_cast<const void*>(&fa::fa_bwd_dq_kernel<HD>));
+}
+
+template <int HD>
+int launch_bwd_stages(const BwdPlan& pl, unsigned stages) {
+  int rc = FA_OK;
+  if ((stages & 1u) && (rc = launch_bwd_prep<HD>(pl)) != FA_OK) return rc;
+  if ((stages & 2u) && (rc = launch_bwd_dkdv<HD>(pl)) != FA_OK) return rc;
+  if ((stages & 4u) && (rc = launch_bwd_dq<HD>(pl)) != FA_OK) return rc;
+  return FA_OK;
 }
 
 // KV-cache forward: R query rows per KV head, S key splits of L keys (L a
@@ -500,7 +555,7 @@ int check_bwd(std::initializer_list<const void*> ptrs, void* workspace, size_t w
   if (B == 0 || N == 0) return -1;  // empty: nothing to launch
   for (const void* p : ptrs)
     if (!aligned16(p)) return FA_ERR_INVALID;
-  if (workspace == nullptr || workspace_bytes < fa_bwd_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
+  if (workspace == nullptr || workspace_bytes < bwd_workspace_bytes(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_INVALID;
   if ((rc = check_device(dev)) != FA_OK) return rc;
   return prepare_kernels(*dev);
@@ -552,58 +607,59 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
   if (B < 0 || N < 0 || Hq < 1 || Hkv < 1 || d < 1 || Hq % Hkv != 0) return 0;
-  const size_t rows_q = static_cast<size_t>(B) * Hq;
-  const size_t kv_acc = bwd_head_split(B, Hq, Hkv, N) > 1 ? 2 * static_cast<size_t>(B) * Hkv * N * d : 0;
-  return sizeof(float) * (2 * rows_q * padded_rows(N) + rows_q * static_cast<size_t>(N) * d + kv_acc);
+  return bwd_workspace_bytes(B, Hq, Hkv, N, d);
 }
+
+}  // extern "C"
+
+namespace {
+
+// Validate, plan every launch of the requested stages, then launch them in
+// stream order. Errors other than a failed launch are returned before any
+// kernel is queued.
+int run_bwd(unsigned stages, std::initializer_list<const void*> ptrs, const void* q, const void* k, const void* v,
+            const void* o, const float* lse, const void* dO, void* dq, void* dk, void* dv, void* ws,
+            size_t ws_bytes, int B, int Hq, int Hkv, int N, int d, float scale, int causal, int dtype,
+            fa_stream_t stream) {
+  int dev = 0;
+  int rc = check_bwd(ptrs, ws, ws_bytes, B, Hq, Hkv, N, d, scale, causal, dtype, &dev);
+  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
+  BwdPlan pl;
+  if ((rc = plan_bwd(&pl, stages, q, k, v, o, lse, dO, dq, dk, dv, ws, B, Hq, Hkv, N, d, scale, causal,
+                     reinterpret_cast<cudaStream_t>(stream))) != FA_OK)
+    return rc;
+  return d == 64 ? launch_bwd_stages<64>(pl, stages) : launch_bwd_stages<128>(pl, stages);
+}
+
+}  // namespace
+
+extern "C" {
 
 int fa_bwd_prep(const void* o, const float* lse, const void* dO, void* workspace, size_t workspace_bytes, int B,
                 int Hq, int Hkv, int N, int d, int dtype, fa_stream_t stream) {
-  int dev = 0;
-  int rc = check_bwd({o, lse, dO}, workspace, workspace_bytes, B, Hq, Hkv, N, d, 1.0f, 0, dtype, &dev);
-  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd_prep<64>(o, lse, dO, workspace, B, Hq, Hkv, N, s)
-                 : launch_bwd_prep<128>(o, lse, dO, workspace, B, Hq, Hkv, N, s);
+  return run_bwd(1u, {o, lse, dO}, nullptr, nullptr, nullptr, o, lse, dO, nullptr, nullptr, nullptr, workspace,
+                 workspace_bytes, B, Hq, Hkv, N, d, 1.0f, 0, dtype, stream);
 }
 
-int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* workspace,
+int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* workspace,
                 size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale, int causal, int dtype,
                 fa_stream_t stream) {
-  int dev = 0;
-  int rc = check_bwd({q, k, v, dO, dk, dv}, workspace, workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype, &dev);
-  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd_main<64>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s)
-                 : launch_bwd_main<128>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s);
+  return run_bwd(2u, {q, k, v, dO, dk, dv}, q, k, v, nullptr, nullptr, dO, nullptr, dk, dv, workspace,
+                 workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype, stream);
 }
 
-int fa_bwd_dq(void* dq, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int dtype,
+int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, void* workspace,
+              size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale, int causal, int dtype,
               fa_stream_t stream) {
-  int dev = 0;
-  int rc = check_bwd({dq}, workspace, workspace_bytes, B, Hq, Hkv, N, d, 1.0f, 0, dtype, &dev);
-  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
-  return launch_bwd_dq(dq, workspace, B, Hq, Hkv, N, d, reinterpret_cast<cudaStream_t>(stream));
+  return run_bwd(4u, {q, k, v, dO, dq}, q, k, v, nullptr, nullptr, dO, dq, nullptr, nullptr, workspace,
+                 workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype, stream);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
            void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
            float scale, int causal, int dtype, fa_stream_t stream) {
-  int dev = 0;
-  int rc = check_bwd({q, k, v, o, lse, dO, dq, dk, dv}, workspace, workspace_bytes, B, Hq, Hkv, N, d, scale, causal,
-                     dtype, &dev);
-  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) {
-    if ((rc = launch_bwd_prep<64>(o, lse, dO, workspace, B, Hq, Hkv, N, s)) != FA_OK) return rc;
-    if ((rc = launch_bwd_main<64>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
-      return rc;
-  } else {
-    if ((rc = launch_bwd_prep<128>(o, lse, dO, workspace, B, Hq, Hkv, N, s)) != FA_OK) return rc;
-    if ((rc = launch_bwd_main<128>(q, k, v, dO, dk, dv, workspace, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
-      return rc;
-  }
-  return launch_bwd_dq(dq, workspace, B, Hq, Hkv, N, d, s);
+  return run_bwd(7u, {q, k, v, o, lse, dO, dq, dk, dv}, q, k, v, o, lse, dO, dq, dk, dv, workspace,
+                 workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype, stream);
 }
 
 }  // extern "C"
@@ -624,8 +680,10 @@ constexpr size_t kNoAllocScratchBytes = FA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
 // Device address of g_noalloc_scratch on the current device, looked up once
-// per device with that device current. In host code the array's name is only
-// a host-side stand-in, never a device address.
+// per device with that device current (the first fa_bwd_noalloc call on the
+// device does it). In host code the array's name is only a host-side
+// stand-in, never a device address. The address is kept for the life of the
+// process, so a device reset after the first call is not supported.
 int noalloc_scratch(int dev, void** out) {
   static std::mutex mu;
   static void* addr[128] = {};
@@ -651,29 +709,17 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   if (rc != FA_OK) return rc;
   if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return FA_OK;
-  if (fa_bwd_workspace_size(B, Hq, Hkv, N, d) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  if (bwd_workspace_bytes(B, Hq, Hkv, N, d) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
   int dev = 0;
   if ((rc = check_device(&dev)) != FA_OK) return rc;
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(dev, &scratch)) != FA_OK) return rc;
-  rc = check_bwd({q, k, v, o, lse, dO, dq, dk, dv}, scratch, kNoAllocScratchBytes, B, Hq, Hkv, N, d, scale, causal,
-                 dtype, &dev);
-  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
-  // Every scratch byte this problem reads is rewritten first (D, LSE and the
-  // dQ accumulator by the prep kernel; the dK/dV accumulators, when the
-  // group's heads are split, by a zeroing kernel before the main kernel), so
-  // what an earlier call left in the array does not matter.
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) {
-    if ((rc = launch_bwd_prep<64>(o, lse, dO, scratch, B, Hq, Hkv, N, s)) != FA_OK) return rc;
-    if ((rc = launch_bwd_main<64>(q, k, v, dO, dk, dv, scratch, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
-      return rc;
-  } else {
-    if ((rc = launch_bwd_prep<128>(o, lse, dO, scratch, B, Hq, Hkv, N, s)) != FA_OK) return rc;
-    if ((rc = launch_bwd_main<128>(q, k, v, dO, dk, dv, scratch, B, Hq, Hkv, N, scale, causal, s)) != FA_OK)
-      return rc;
-  }
-  return launch_bwd_dq(dq, scratch, B, Hq, Hkv, N, d, s);
+  // Every scratch byte this problem reads is rewritten first (D and LSE by
+  // the prep kernel; the dK/dV accumulators, when the group's heads are
+  // split, by a zeroing kernel before the dK/dV kernel), so what an earlier
+  // call left in the array does not matter.
+  return run_bwd(7u, {q, k, v, o, lse, dO, dq, dk, dv}, q, k, v, o, lse, dO, dq, dk, dv, scratch,
+                 kNoAllocScratchBytes, B, Hq, Hkv, N, d, scale, causal, dtype, stream);
 }
 
 size_t fa_fwd_kvcache_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d) {

@@ -89,6 +89,23 @@ FA_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& w) {
   }
 }
 
+// Wait for the phase with parity `parity` of barrier `bar` regardless of the
+// CTA's abort flag, bounded by `timeout_ns`: used on the way out of a kernel
+// to make sure no copy or MMA the CTA issued is still in flight before its
+// shared and tensor memory are released. Returns false (and records a
+// timeout) if the limit runs out.
+FA_DEV bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > timeout_ns) {
+      atomicCAS(&g_status, 0, kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
 // mbar_wait for a whole warp whose lanes must stay converged (collective
 // tcgen05 loads follow): true only if every lane's wait succeeded.
 FA_DEV bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl& w) {

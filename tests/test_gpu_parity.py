@@ -4,9 +4,12 @@ Tolerances: float32 inputs, O and LSE max-abs <= 1e-5; bf16 inputs with fp32
 accumulation, O max-abs <= 2e-2 and LSE max-abs <= 1e-3; gradients dQ, dK, dV
 relative Frobenius error <= 2e-2. Inputs are the seeded synthetic tensors of
 ``exact_io_aware_61_b200.inputs``; the oracle gets the same values in fp64.
-Full-size workloads are checked on sampled rows (forward) or sampled heads
-(backward) that the oracle computes one by one, plus properties that hold at
-any size.
+Full-size workloads are checked against the oracle head by head (every row
+of the benchmark forward, every head of the training backward) or on sampled
+rows and whole KV-head groups where a full check would take too long, plus
+properties that hold at any size. Every output is written into a view of a
+larger, canary-filled buffer, and the canaries are checked after each call
+(``tests/guarded.py``).
 """
 
 import numpy as np
@@ -15,6 +18,7 @@ import torch
 
 import oracle.attention as ORACLE
 from exact_io_aware_61_b200 import inputs as INP
+from tests.guarded import Guarded, check_all
 
 pytestmark = pytest.mark.gpu
 
@@ -37,11 +41,18 @@ def _to_dev(t):
 
 
 def _run_fwd(fa, inp, causal, scale):
+    """fa_fwd into canary-guarded O and LSE (pre-filled with NaN, so a row the
+    kernel never writes fails the comparison and a store outside them fails
+    the guard check)."""
     q, k, v = (_to_dev(inp[n]) for n in ("q", "k", "v"))
-    o, lse = fa.forward(q, k, v, causal=causal, scale=scale)
+    B, Hq, N, d = q.shape
+    go = Guarded(q.shape, q.dtype, fill=float("nan"))
+    gl = Guarded((B, Hq, N), torch.float32, fill=float("nan"))
+    fa.fa_fwd(q, k, v, go.t, gl.t, causal, scale)
     torch.cuda.synchronize()
     assert fa.fa_last_device_status() == fa.FA_OK
-    return o, lse
+    check_all(("O", go), ("LSE", gl))
+    return go.t, gl.t
 
 
 def _rel_fro(a, b):
@@ -110,12 +121,33 @@ def _sample_rows(N, rng, n_random=24):
     return sorted(rows)
 
 
+def test_fwd_causal_bf16_b2_h32_n8192_d128_all_rows(fa):
+    """The benchmark forward (B=2, H=32, N=8192, d=128, causal): every row of
+    every head against the full oracle, one head at a time."""
+    w = INP.WORKLOADS["fwd_causal_bf16_b2_h32_n8192_d128"]
+    inp = INP.workload_inputs(w, seed=1003)
+    o, lse = _run_fwd(fa, inp, True, w.scale)
+    o_h, lse_h = o.float().cpu().numpy(), lse.cpu().numpy()
+    q, k, v = (inp[n].float().numpy() for n in "qkv")
+    worst_o = worst_l = 0.0
+    for b in range(w.B):
+        for h in range(w.Hq):
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            ro, rl = ORACLE.attention_forward(q[sl], k[sl], v[sl], w.scale, True)
+            worst_o = max(worst_o, float(np.max(np.abs(o_h[sl] - ro))))
+            worst_l = max(worst_l, float(np.max(np.abs(lse_h[sl] - rl))))
+    assert worst_o <= O_TOL_BF16, worst_o
+    assert worst_l <= LSE_TOL_BF16, worst_l
+
+
 @pytest.mark.parametrize("name", [
-    "fwd_causal_bf16_b2_h32_n8192_d128",
     "gqa_causal_bf16_b1_h32_kv8_n16384_d128",
     "gqa_causal_bf16_b1_h16_kv4_n8192_d256",
 ])
 def test_fwd_bf16_full_size_sampled_rows(fa, name):
+    """The grouped-query workloads: sampled rows of every head (tile
+    boundaries, the first and last rows, random rows), plus every row of the
+    last KV head's group in blocks of 2048 queries."""
     w = INP.WORKLOADS[name]
     inp = INP.workload_inputs(w, seed=1000 + len(name))
     o, lse = _run_fwd(fa, inp, True, w.scale)
@@ -123,12 +155,17 @@ def test_fwd_bf16_full_size_sampled_rows(fa, name):
     q, k, v = (inp[n].float().numpy() for n in "qkv")
     rng = np.random.default_rng(7)
     worst_o = worst_l = 0.0
+    g = w.Hq // w.Hkv
     for b in range(w.B):
         for h in range(w.Hq):
-            rows = _sample_rows(w.N, rng)
-            ro, rl = ORACLE.attention_forward_rows(q, k, v, w.scale, True, b, h, rows)
-            worst_o = max(worst_o, float(np.max(np.abs(o_h[b, h, rows] - ro))))
-            worst_l = max(worst_l, float(np.max(np.abs(lse_h[b, h, rows] - rl))))
+            if h >= w.Hq - g:  # the last group: all rows
+                blocks = [list(range(r, min(r + 2048, w.N))) for r in range(0, w.N, 2048)]
+            else:
+                blocks = [_sample_rows(w.N, rng)]
+            for rows in blocks:
+                ro, rl = ORACLE.attention_forward_rows(q, k, v, w.scale, True, b, h, rows)
+                worst_o = max(worst_o, float(np.max(np.abs(o_h[b, h, rows] - ro))))
+                worst_l = max(worst_l, float(np.max(np.abs(lse_h[b, h, rows] - rl))))
     assert worst_o <= O_TOL_BF16, worst_o
     assert worst_l <= LSE_TOL_BF16, worst_l
     assert np.all(np.isfinite(o_h)) and np.all(np.isfinite(lse_h))
@@ -143,18 +180,28 @@ def test_fwd_bf16_deterministic(fa):
 
 # ----------------------------------------------------------------- backward
 
-def _run_bwd(fa, inp, causal, scale):
+def _run_bwd(fa, inp, causal, scale, return_fwd=False):
+    """fa_fwd, then fa_bwd into canary-guarded dQ, dK, dV and workspace."""
     q, k, v, do = (_to_dev(inp[n]) for n in ("q", "k", "v", "do"))
-    o, lse = fa.forward(q, k, v, causal=causal, scale=scale)
-    dq, dk, dv = fa.backward(q, k, v, o, lse, do, causal=causal, scale=scale)
+    o, lse = _run_fwd(fa, inp, causal, scale)
+    B, Hq, N, d = q.shape
+    gq = Guarded(q.shape, q.dtype, fill=float("nan"))
+    gk = Guarded(k.shape, k.dtype, fill=float("nan"))
+    gv = Guarded(v.shape, v.dtype, fill=float("nan"))
+    gw = Guarded((max(fa.fa_bwd_workspace_size(B, Hq, k.shape[1], N, d), 16),), torch.uint8)
+    fa.fa_bwd(q, k, v, o, lse, do, gq.t, gk.t, gv.t, gw.t, causal, scale)
     torch.cuda.synchronize()
     assert fa.fa_last_device_status() == fa.FA_OK
-    return dq, dk, dv
+    check_all(("dQ", gq), ("dK", gk), ("dV", gv), ("workspace", gw))
+    if return_fwd:
+        return gq.t, gk.t, gv.t, o, lse
+    return gq.t, gk.t, gv.t
 
 
 BWD_SHAPES = [
     (1, 1, 1, 1, 64), (1, 2, 2, 100, 64), (1, 2, 2, 128, 128), (2, 2, 2, 257, 128),
     (1, 4, 2, 300, 64), (1, 4, 1, 384, 128), (1, 2, 2, 1000, 128), (2, 6, 3, 513, 64),
+    (1, 8, 1, 2048, 128), (2, 4, 1, 1500, 64),  # MQA: the group's heads split over CTAs
 ]
 
 
@@ -172,22 +219,68 @@ def test_bwd_bf16_shapes(fa, shape, causal):
 
 
 def test_bwd_train_causal_b2_h16_n4096_d128(fa):
+    """The training workload (B=2, H=16, N=4096, d=128, causal): dQ, dK and dV
+    of all 32 (batch, head) pairs against the full fp64 analytic backward."""
     w = INP.WORKLOADS["train_causal_bf16_b2_h16_n4096_d128"]
     inp = INP.workload_inputs(w, seed=1005)
     dq, dk, dv = _run_bwd(fa, inp, True, w.scale)
     dq_h, dk_h, dv_h = (INP.as_f64(t) for t in (dq, dk, dv))
-    # property at full size: every row of P sums to one, so sum_j dV_j = sum_i dO_i
-    do = INP.as_f64(inp["do"])
-    lhs, rhs = dv_h.sum(axis=2), do.sum(axis=2)
-    assert _rel_fro(lhs, rhs) <= GRAD_TOL
-    # full oracle on sampled heads
-    q, k, v = (INP.as_f64(inp[n]) for n in "qkv")
-    for b, h in ((0, 0), (0, 7), (1, 3), (1, 15)):
+    q, k, v, do = (inp[n].float().numpy() for n in ("q", "k", "v", "do"))
+    for b in range(w.B):
+        for h in range(w.Hq):
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            rq, rk, rv, _ = ORACLE.attention_backward(q[sl], k[sl], v[sl], do[sl], w.scale, True)
+            for name, got, ref in (("dq", dq_h[sl], rq), ("dk", dk_h[sl], rk), ("dv", dv_h[sl], rv)):
+                err = _rel_fro(got, ref)
+                assert err <= GRAD_TOL, (name, b, h, err)
+
+
+def _group_identities(dk_h, dv_h, do_h, Hq, Hkv):
+    """Checks that hold at any size, for every (batch, KV head):
+    sum_j dV_j = sum over the group's query heads of sum_i dO_i (every row of P
+    sums to one), and sum_j dK_j = 0 (every row of dS = P * (dP - D) sums to
+    zero, since D_i = sum_j P_ij dP_ij). The second is measured against the
+    size of the rows it sums: rounding alone leaves about 2^-9 of it."""
+    g = Hq // Hkv
+    for b in range(dk_h.shape[0]):
+        for hk in range(Hkv):
+            lhs = dv_h[b, hk].sum(axis=0)
+            rhs = do_h[b, hk * g:(hk + 1) * g].sum(axis=(0, 1))
+            assert _rel_fro(lhs, rhs) <= GRAD_TOL, ("sum dV", b, hk)
+            zero = np.linalg.norm(dk_h[b, hk].sum(axis=0))
+            scale = np.sqrt(np.sum(dk_h[b, hk] ** 2))
+            assert zero <= GRAD_TOL * scale, ("sum dK", b, hk, zero / scale)
+
+
+def test_bwd_causal_b2_h32_n8192_d128(fa):
+    """The benchmark backward (B=2, H=32, N=8192, d=128, causal), the shape
+    bench.py times. Full fp64 dQ, dK, dV on one head from every group of 8
+    consecutive (batch, head) pairs (8 heads, the first and last included);
+    the dV and dK identities on every head; exact dQ on sampled rows of every
+    head."""
+    B, H, N, d = 2, 32, 8192, 128
+    scale = d ** -0.5
+    inp = INP.make_inputs(B, H, H, N, d, "bf16", seed=1003, grad=True)
+    dq, dk, dv = _run_bwd(fa, inp, True, scale)
+    dq_h, dk_h, dv_h = (INP.as_f64(t) for t in (dq, dk, dv))
+    q, k, v, do = (inp[n].float().numpy() for n in ("q", "k", "v", "do"))
+    for grp in range(B * H // 8):
+        bh = 8 * grp + (grp * 3) % 8 if grp < B * H // 8 - 1 else B * H - 1
+        b, h = divmod(bh, H)
         sl = (slice(b, b + 1), slice(h, h + 1))
-        rq, rk, rv, _ = ORACLE.attention_backward(q[sl], k[sl], v[sl], do[sl], w.scale, True)
+        rq, rk, rv, _ = ORACLE.attention_backward(q[sl], k[sl], v[sl], do[sl], scale, True)
         for name, got, ref in (("dq", dq_h[sl], rq), ("dk", dk_h[sl], rk), ("dv", dv_h[sl], rv)):
             err = _rel_fro(got, ref)
             assert err <= GRAD_TOL, (name, b, h, err)
+    _group_identities(dk_h, dv_h, do.astype(np.float64), H, H)
+    rng = np.random.default_rng(13)
+    worst = 0.0
+    for b in range(B):
+        for h in range(H):
+            rows = _sample_rows(N, rng, n_random=6)
+            rq, _, _ = ORACLE.attention_backward_rows(q, k, v, do, scale, True, b, h, rows)
+            worst = max(worst, _rel_fro(dq_h[b, h, rows], rq))
+    assert worst <= GRAD_TOL, worst
 
 
 def test_bwd_gqa_causal_b1_h8_kv2_n4096_d128_full_group(fa):
@@ -208,29 +301,39 @@ def test_bwd_gqa_causal_b1_h8_kv2_n4096_d128_full_group(fa):
 
 
 def test_bwd_gqa_causal_b1_h32_kv8_n16384_d128(fa):
-    """GQA backward at the 16k-token GQA workload: exact dQ on sampled rows of
-    every query head, and for every KV head the identity sum_j dV_j =
-    sum over the group's heads of sum_i dO_i (each row of P sums to one)."""
+    """GQA backward at the 16k-token GQA workload: dQ, dK and dV of the last KV
+    head's group in full (dK and dV as the sum of the oracle's per-row-block
+    shares over all 16384 queries of its four query heads), the dV and dK
+    identities on every KV head, and exact dQ on sampled rows of every query
+    head."""
     w = INP.WORKLOADS["gqa_causal_bf16_b1_h32_kv8_n16384_d128"]
     inp = INP.make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, "bf16", seed=16384 + 32, grad=True)
     dq, dk, dv = _run_bwd(fa, inp, True, w.scale)
-    dq_h = dq.float().cpu().numpy()
-    dv_h = dv.float().cpu().numpy().astype(np.float64)
+    dq_h, dk_h, dv_h = (INP.as_f64(t) for t in (dq, dk, dv))
     q, k, v, do = (inp[n].float().numpy() for n in ("q", "k", "v", "do"))
     g = w.Hq // w.Hkv
-    for hk in range(w.Hkv):
-        lhs = dv_h[0, hk].sum(axis=0)
-        rhs = do[0, hk * g:(hk + 1) * g].astype(np.float64).sum(axis=(0, 1))
-        assert _rel_fro(lhs, rhs) <= GRAD_TOL, ("dv sum", hk)
+    hk = w.Hkv - 1
+    rk = np.zeros((w.N, w.d))
+    rv = np.zeros((w.N, w.d))
+    for h in range(hk * g, (hk + 1) * g):
+        rq = np.zeros((w.N, w.d))
+        for r0 in range(0, w.N, 2048):
+            rows = list(range(r0, min(r0 + 2048, w.N)))
+            dq_rows, dk_part, dv_part = ORACLE.attention_backward_rows(q, k, v, do, w.scale, True, 0, h, rows)
+            rq[rows] = dq_rows
+            rk += dk_part
+            rv += dv_part
+        assert _rel_fro(dq_h[0, h], rq) <= GRAD_TOL, ("dq", h)
+    assert _rel_fro(dk_h[0, hk], rk) <= GRAD_TOL, "dk"
+    assert _rel_fro(dv_h[0, hk], rv) <= GRAD_TOL, "dv"
+    _group_identities(dk_h, dv_h, do.astype(np.float64), w.Hq, w.Hkv)
     rng = np.random.default_rng(11)
     worst = 0.0
     for h in range(w.Hq):
         rows = _sample_rows(w.N, rng, n_random=6)
         rq, _, _ = ORACLE.attention_backward_rows(q, k, v, do, w.scale, True, 0, h, rows)
-        worst = max(worst, _rel_fro(dq_h[0, h, rows].astype(np.float64), rq))
+        worst = max(worst, _rel_fro(dq_h[0, h, rows], rq))
     assert worst <= GRAD_TOL, worst
-    assert np.all(np.isfinite(dq_h)) and np.all(np.isfinite(dv_h))
-    assert torch.isfinite(dk.float()).all()
 
 
 # ------------------------------------------------------- KV-cache forward
@@ -246,6 +349,21 @@ KVCACHE_SHAPES = [  # (B, Hq, Hkv, Nq, Nk, d)
 ]
 
 
+def _run_kvcache(fa, q, k, v, causal, scale):
+    """fa_fwd_kvcache into canary-guarded O, LSE and workspace."""
+    q, k, v = (_to_dev(t) for t in (q, k, v))
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    go = Guarded(q.shape, q.dtype, fill=float("nan"))
+    gl = Guarded((B, Hq, Nq), torch.float32, fill=float("nan"))
+    gw = Guarded((max(fa.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, Nq, Nk, d), 16),), torch.uint8)
+    fa.fa_fwd_kvcache(q, k, v, go.t, gl.t, gw.t, causal, scale)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.FA_OK
+    check_all(("O", go), ("LSE", gl), ("workspace", gw))
+    return go.t, gl.t
+
+
 def _kvcache_inputs(B, Hq, Hkv, Nq, Nk, d, seed):
     # the new queries are the last Nq rows of a seeded square problem
     inp = INP.make_inputs(B, Hq, Hkv, Nk, d, "bf16", seed=seed)
@@ -257,9 +375,7 @@ def _kvcache_inputs(B, Hq, Hkv, Nq, Nk, d, seed):
 def test_fwd_kvcache_bf16(fa, shape, causal):
     B, Hq, Hkv, Nq, Nk, d = shape
     q, k, v = _kvcache_inputs(B, Hq, Hkv, Nq, Nk, d, seed=Nk + 7 * Nq + d)
-    o, lse = fa.forward_kvcache(_to_dev(q), _to_dev(k), _to_dev(v), causal=causal, scale=d ** -0.5)
-    torch.cuda.synchronize()
-    assert fa.fa_last_device_status() == fa.FA_OK
+    o, lse = _run_kvcache(fa, q, k, v, causal, d ** -0.5)
     ro, rl = ORACLE.attention_forward_kvcache(INP.as_f64(q), INP.as_f64(k), INP.as_f64(v), d ** -0.5, causal)
     assert np.max(np.abs(INP.as_f64(o) - ro)) <= O_TOL_BF16
     assert np.max(np.abs(INP.as_f64(lse) - rl)) <= LSE_TOL_BF16
@@ -273,9 +389,7 @@ def test_fwd_kvcache_decode_b8_h32_kv8_nk32768_d128(fa):
     q = torch.randn((B, Hq, Nq, d), generator=g).to(torch.bfloat16)
     k = torch.randn((B, Hkv, Nk, d), generator=g).to(torch.bfloat16)
     v = torch.randn((B, Hkv, Nk, d), generator=g).to(torch.bfloat16)
-    o, lse = fa.forward_kvcache(_to_dev(q), _to_dev(k), _to_dev(v), causal=True, scale=d ** -0.5)
-    torch.cuda.synchronize()
-    assert fa.fa_last_device_status() == fa.FA_OK
+    o, lse = _run_kvcache(fa, q, k, v, True, d ** -0.5)
     ro, rl = ORACLE.attention_forward_kvcache(INP.as_f64(q), INP.as_f64(k), INP.as_f64(v), d ** -0.5, True)
     assert np.max(np.abs(INP.as_f64(o) - ro)) <= O_TOL_BF16
     assert np.max(np.abs(INP.as_f64(lse) - rl)) <= LSE_TOL_BF16
