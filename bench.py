@@ -2,10 +2,10 @@
 """Throughput of exact causal attention, forward + backward, bf16, on B200.
 
 One step is the whole hot path over one batch: ``fa_fwd`` (O, LSE), then the
-three backward stages ``fa_bwd_prep`` (D and the padded LSE), ``fa_bwd_dkdv``
-(key-side recompute: dK, dV) and ``fa_bwd_dq`` (query-side recompute: dQ),
-on B=2, Hq=Hkv=32, N=8192, d=128, causal, synthetic N(0,1) inputs rounded to
-bf16. FLOPs follow the usual convention: forward 4*B*Hq*N^2*d, halved when
+three backward stages ``fa_bwd_prep`` (D, padded LSE, zeroed dQ accumulator),
+``fa_bwd_main`` (recompute, dK, dV, dQ accumulation) and ``fa_bwd_dq``
+(dQ to bf16), on B=2, Hq=Hkv=32, N=8192, d=128, causal, synthetic N(0,1)
+inputs rounded to bf16. FLOPs follow the usual convention: forward 4*B*Hq*N^2*d, halved when
 causal; backward 2.5 times the forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -60,16 +60,13 @@ def bwd_flops(B, Hq, N, d, causal):
 
 
 def kernel_flops(B, Hq, N, d, causal):
-    """Algorithmic FLOPs credited to each kernel, and the FLOPs it executes.
+    """Algorithmic FLOPs credited to each tensor-core kernel, and the FLOPs it executes.
 
-    Each of the backward's five products (S, dP, dV, dK, dQ) costs half the
-    forward. The dK/dV kernel computes S^T, dP^T, dV and dK: four products,
-    all of them the method's own work. The dQ kernel computes S, dP and dQ;
-    only dQ is new work, S and dP are computed a second time so that dQ can be
-    accumulated on chip. The credited FLOPs add up to the convention's 2.5x.
+    The backward's five products (S, dP, dV, dK, dQ) all run in the main
+    kernel, each once: 2.5 times the forward, the convention's figure.
     """
     f = fwd_flops(B, Hq, N, d, causal)
-    return {"fwd": (f, f), "bwd_dkdv": (2.0 * f, 2.0 * f), "bwd_dq": (0.5 * f, 1.5 * f)}
+    return {"fwd": (f, f), "bwd_main": (2.5 * f, 2.5 * f)}
 
 
 def algorithmic_bytes(B, Hq, Hkv, N, d):
@@ -79,9 +76,9 @@ def algorithmic_bytes(B, Hq, Hkv, N, d):
     rows = B * Hq * N * 4
     return {
         "fwd": q + 2 * kv + q + rows,                     # read Q, K, V; write O, LSE
-        "bwd_prep": 2 * q + rows + 2 * rows,              # read O, dO, LSE; write D, LSE2
-        "bwd_dkdv": 2 * q + 2 * kv + 2 * rows + 2 * kv,   # read Q, dO, K, V, LSE2, D; write dK, dV
-        "bwd_dq": 2 * q + 2 * kv + 2 * rows + q,          # read Q, dO, K, V, LSE2, D; write dQ
+        "bwd_prep": 2 * q + rows + 2 * rows + 2 * q,      # read O, dO, LSE; write D, LSE2, zero dQacc (f32)
+        "bwd_main": 2 * q + 2 * kv + 2 * rows + 2 * kv + 2 * q * 2,  # read Q,dO,K,V,LSE2,D; write dK,dV; dQacc add
+        "bwd_dq": 2 * q + q,                              # read dQacc (f32), write dQ
     }
 
 
@@ -277,9 +274,16 @@ def run_ours(args, rank, world, local):
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     fa.load()
-    B, Hq, Hkv, N, d = (SHAPE[k] for k in ("B", "Hq", "Hkv", "N", "d"))
+    from exact_io_aware_61_b200.shard import pair_range
+
+    # The job is world x the benchmark workload; its (batch, KV head) pairs are
+    # split over the ranks in contiguous ranges (no collective on the data
+    # path), so every rank runs the benchmark shape on its own slice.
+    Hq, Hkv, N, d = (SHAPE[k] for k in ("Hq", "Hkv", "N", "d"))
+    shard = pair_range(SHAPE["B"] * world, Hq, Hkv, rank, world)
+    B, Hq, Hkv = shard.local_shape()
     scale = d ** -0.5
-    host = inp_mod.make_inputs(B, Hq, Hkv, N, d, "bf16", SEED + rank, grad=True)
+    host = inp_mod.make_inputs(B, Hq, Hkv, N, d, "bf16", SEED + shard.p0, grad=True)
     q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
@@ -296,10 +300,10 @@ def run_ours(args, rank, world, local):
         fa.fa_bwd_prep(o, lse, do, ws, Hkv, stream)
         if ev is not None:
             ev[2].record(stream)
-        fa.fa_bwd_dkdv(q, k, v, do, dk, dv, ws, CAUSAL, scale, stream)
+        fa.fa_bwd_main(q, k, v, do, dk, dv, ws, CAUSAL, scale, stream)
         if ev is not None:
             ev[3].record(stream)
-        fa.fa_bwd_dq(q, k, v, do, dq, ws, CAUSAL, scale, stream)
+        fa.fa_bwd_dq(dq, ws, Hkv, stream)
         if ev is not None:
             ev[4].record(stream)
 
@@ -329,14 +333,14 @@ def run_ours(args, rank, world, local):
 
     elapsed_ms = start.elapsed_time(end)
     per_kernel = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in events)
-                  for i, name in enumerate(("fwd", "bwd_prep", "bwd_dkdv", "bwd_dq"))}
+                  for i, name in enumerate(("fwd", "bwd_prep", "bwd_main", "bwd_dq"))}
     max_ms = max_over_ranks(elapsed_ms, world, dev)
 
     f_fwd = fwd_flops(B, Hq, N, d, CAUSAL)
     f_bwd = bwd_flops(B, Hq, N, d, CAUSAL)
     step_flops = f_fwd + f_bwd
     value = world * step_flops * args.steps / (max_ms / 1e3) / 1e12
-    bwd_ms = per_kernel["bwd_prep"] + per_kernel["bwd_dkdv"] + per_kernel["bwd_dq"]
+    bwd_ms = per_kernel["bwd_prep"] + per_kernel["bwd_main"] + per_kernel["bwd_dq"]
 
     # forward alone: its own timed region (no backward kernels in between)
     fwd_only = None
@@ -390,8 +394,8 @@ def run_ours(args, rank, world, local):
             comp.wait_event(downloaded[s])  # step i-2's outputs have left this set
             fa.fa_fwd(b["q"], b["k"], b["v"], b["o"], b["lse"], CAUSAL, scale, comp)
             fa.fa_bwd_prep(b["o"], b["lse"], b["do"], b["ws"], Hkv, comp)
-            fa.fa_bwd_dkdv(b["q"], b["k"], b["v"], b["do"], b["dk"], b["dv"], b["ws"], CAUSAL, scale, comp)
-            fa.fa_bwd_dq(b["q"], b["k"], b["v"], b["do"], b["dq"], b["ws"], CAUSAL, scale, comp)
+            fa.fa_bwd_main(b["q"], b["k"], b["v"], b["do"], b["dk"], b["dv"], b["ws"], CAUSAL, scale, comp)
+            fa.fa_bwd_dq(b["dq"], b["ws"], Hkv, comp)
             computed[s].record(comp)
             down.wait_event(computed[s])
             with torch.cuda.stream(down):
@@ -440,7 +444,7 @@ def run_ours(args, rank, world, local):
     kf = kernel_flops(B, Hq, N, d, CAUSAL)
     src_hash = kernel_source_hash()
     names = {"fwd": f"fa_fwd_bf16_2tile_kernel<{d}>", "bwd_prep": f"fa_bwd_prep_kernel<{d}>",
-             "bwd_dkdv": f"fa_bwd_dkdv_kernel<{d}>", "bwd_dq": f"fa_bwd_dq_kernel<{d}>"}
+             "bwd_main": f"fa_bwd2_main_kernel<{d}>", "bwd_dq": "fa_bwd_dq_kernel"}
     kernels = {}
     for name, ms in per_kernel.items():
         e = {"kernel": names[name], "ms": round(ms, 4), "gbs": round(nbytes[name] / ms / 1e6, 1)}
@@ -476,7 +480,8 @@ def run_ours(args, rank, world, local):
         "dtype": "bf16",
         "data": "synthetic: i.i.d. N(0,1) rounded to bf16, seeded",
         "config": {"workload": WORKLOAD_NAME, "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": CAUSAL,
-                   "parallelism": f"{world} independent replicas (one per GPU), no collective",
+                   "parallelism": f"(batch, KV head) pairs of a {SHAPE['B'] * world}-batch job split over {world} "
+                                  f"rank(s), {shard.pairs} pairs each, no collective on the data path",
                    "l2": "no flush: every step streams > 1 GB and each of Q, K, V, O, dO is 134 MB (> 126 MB L2)"},
         "fwd_tflops": round(f_fwd / per_kernel["fwd"] / 1e9, 2),
         "bwd_tflops": round(f_bwd / bwd_ms / 1e9, 2),
@@ -490,7 +495,7 @@ def run_ours(args, rank, world, local):
                         "spec_tflops": SPEC_BF16_TFLOPS,
                         "spec_source": "vendor dense bf16 figure (the 2:4-sparse figure halved)"},
         "hbm_gbs": {"fwd": kernels["fwd"]["gbs"],
-                    "bwd": round(sum(nbytes[n] for n in ("bwd_prep", "bwd_dkdv", "bwd_dq")) / bwd_ms / 1e6, 1),
+                    "bwd": round(sum(nbytes[n] for n in ("bwd_prep", "bwd_main", "bwd_dq")) / bwd_ms / 1e6, 1),
                     "peak_gbs": hbm},
         "kernels": kernels,
         "roofline": {"kernel": names[dominant], "bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf,

@@ -19,7 +19,7 @@ from ._lib import (  # noqa: F401
     FAError,
     backward,
     fa_bwd,
-    fa_bwd_dkdv,
+    fa_bwd_main,
     fa_bwd_dq,
     fa_bwd_noalloc,
     fa_bwd_prep,

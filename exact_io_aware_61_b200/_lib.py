@@ -24,7 +24,7 @@ EXPORTED = (
     "fa_fwd",
     "fa_bwd",
     "fa_bwd_prep",
-    "fa_bwd_dkdv",
+    "fa_bwd_main",
     "fa_bwd_dq",
     "fa_bwd_noalloc",
     "fa_bwd_workspace_size",
@@ -64,9 +64,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_bwd.restype = i
         lib.fa_bwd_prep.argtypes = [vp, vp, vp, vp, sz, i, i, i, i, i, i, vp]
         lib.fa_bwd_prep.restype = i
-        lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp]
-        lib.fa_bwd_dkdv.restype = i
-        lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp]
+        lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp]
+        lib.fa_bwd_main.restype = i
+        lib.fa_bwd_dq.argtypes = [vp, vp, sz, i, i, i, i, i, i, vp]
         lib.fa_bwd_dq.restype = i
         lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
         lib.fa_bwd_noalloc.restype = i
@@ -158,7 +158,7 @@ def _ws(workspace):
 
 
 def fa_bwd_prep(o, lse, do, workspace, Hkv: int, stream=None) -> None:
-    """Stage 1 of ``fa_bwd``: D and the padded log2 LSE in ``workspace``."""
+    """Stage 1 of ``fa_bwd``: D, padded log2 LSE and a zeroed dQ accumulator in ``workspace``."""
     B, Hq, N, d = o.shape
     ws, nbytes = _ws(workspace)
     rc = load().fa_bwd_prep(_ptr(o), _ptr(lse), _ptr(do), ws, nbytes, B, Hq, Hkv, N, d, _dtype_code(o),
@@ -167,23 +167,23 @@ def fa_bwd_prep(o, lse, do, workspace, Hkv: int, stream=None) -> None:
         raise FAError(rc, "fa_bwd_prep")
 
 
-def fa_bwd_dkdv(q, k, v, do, dk, dv, workspace, causal: bool, scale: float, stream=None) -> None:
-    """Stage 2 of ``fa_bwd``: the key-side recompute kernel (dK, dV)."""
+def fa_bwd_main(q, k, v, do, dk, dv, workspace, causal: bool, scale: float, stream=None) -> None:
+    """Stage 2 of ``fa_bwd``: the recompute kernel (dK, dV, and dQ into the accumulator)."""
     B, Hq, N, d = q.shape
     ws, nbytes = _ws(workspace)
-    rc = load().fa_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk), _ptr(dv), ws, nbytes, B, Hq,
+    rc = load().fa_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk), _ptr(dv), ws, nbytes, B, Hq,
                             k.shape[1], N, d, float(scale), int(bool(causal)), _dtype_code(q),
                             ctypes.c_void_p(_stream_ptr(stream)))
     if rc != FA_OK:
-        raise FAError(rc, "fa_bwd_dkdv")
+        raise FAError(rc, "fa_bwd_main")
 
 
-def fa_bwd_dq(q, k, v, do, dq, workspace, causal: bool, scale: float, stream=None) -> None:
-    """Stage 3 of ``fa_bwd``: the query-side recompute kernel (dQ)."""
-    B, Hq, N, d = q.shape
+def fa_bwd_dq(dq, workspace, Hkv: int, stream=None) -> None:
+    """Stage 3 of ``fa_bwd``: f32 accumulator -> bf16 ``dq``."""
+    B, Hq, N, d = dq.shape
     ws, nbytes = _ws(workspace)
-    rc = load().fa_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), ws, nbytes, B, Hq, k.shape[1], N, d,
-                          float(scale), int(bool(causal)), _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    rc = load().fa_bwd_dq(_ptr(dq), ws, nbytes, B, Hq, Hkv, N, d, _dtype_code(dq),
+                          ctypes.c_void_p(_stream_ptr(stream)))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd_dq")
 

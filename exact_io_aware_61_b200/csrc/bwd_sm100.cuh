@@ -1,11 +1,12 @@
-// bwd_sm100.cuh -- the memory-bound stages around the backward kernels
-// (bwd_dkdv_sm100.cuh, bwd_dq_sm100.cuh):
-//   fa_bwd_prep_kernel     D = rowsum(dO * O) and LSE * log2(e) into
-//                          128-row-padded workspace rows (+inf / 0 in the
-//                          padding, so padded queries get zero weight)
-//   fa_f32_to_bf16_kernel  f32 accumulator -> bf16 (dK, dV when the
-//                          backward splits a group's heads over CTAs)
-//   fa_zero_f32_kernel     zero an f32 accumulator
+// bwd_sm100.cuh -- the memory-bound stages around the backward main kernel
+// (bwd2_sm100.cuh):
+//   fa_bwd_prep_kernel   D = rowsum(dO * O) and LSE * log2(e) into
+//                        128-row-padded workspace rows (+inf / 0 in the
+//                        padding, so padded queries get zero weight), and
+//                        zeroing of the f32 dQ accumulator
+//   fa_bwd_dq_kernel     f32 accumulator -> bf16 (dQ; dK, dV when the
+//                        backward splits a group's heads over CTAs)
+//   fa_zero_f32_kernel   zero an f32 accumulator
 #pragma once
 
 #include <cuda.h>
@@ -22,6 +23,7 @@ struct BwdPrepParams {
   const float* lse;
   float* ws_delta;  // [B*Hq][Npad]
   float* ws_lse2;   // [B*Hq][Npad]
+  float* dq_acc;    // [B*Hq][N][d]
   int N, Npad;
 };
 
@@ -40,6 +42,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p)
     const size_t off = (bh * p.N + row) * HD + sub * PER;
     const uint4* o4 = reinterpret_cast<const uint4*>(p.o + off);
     const uint4* d4 = reinterpret_cast<const uint4*>(p.dO + off);
+    float4* z4 = reinterpret_cast<float4*>(p.dq_acc + off);
 #pragma unroll
     for (int i = 0; i < PER / 8; ++i) {
       const uint4 a = o4[i], g = d4[i];
@@ -50,6 +53,8 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p)
         acc = fmaf(bf16_lo(av[t]), bf16_lo(gv[t]), acc);
         acc = fmaf(bf16_hi(av[t]), bf16_hi(gv[t]), acc);
       }
+      z4[2 * i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z4[2 * i + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
@@ -62,18 +67,18 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p)
   }
 }
 
-// ------------------------------------------------------- f32 -> bf16
+// ------------------------------------------------------------ dQ convert
 
-// grid-stride over float4 groups of the accumulator: out = bf16(acc).
-__global__ void __launch_bounds__(256) fa_f32_to_bf16_kernel(const float* __restrict__ acc,
-                                                             __nv_bfloat16* __restrict__ out, size_t n4) {
+// grid-stride over float4 groups of the accumulator: dq = bf16(acc).
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ acc,
+                                                        __nv_bfloat16* __restrict__ dq, size_t n4) {
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const float4 v = reinterpret_cast<const float4*>(acc)[i];
     uint2 w;
     w.x = pack_bf16x2(v.x, v.y);
     w.y = pack_bf16x2(v.z, v.w);
-    reinterpret_cast<uint2*>(out)[i] = w;
+    reinterpret_cast<uint2*>(dq)[i] = w;
   }
 }
 

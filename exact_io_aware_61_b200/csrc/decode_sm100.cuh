@@ -134,10 +134,12 @@ __global__ void __launch_bounds__(256, (DecodeCfg<HD, RB>::MIN_BLOCKS))
       tma_load_3d(sV + s * C::TILE_BYTES + c * (64 * 128), &tm_v, bar, c * 64, k_begin + t * BK, bhkv);
     }
   };
+  int issued = 0;  // tiles whose loads thread 0 has issued
   if (tid == 0) {
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     for (int t = 0; t < min(ST, n_tiles); ++t) issue(t);
+    issued = min(ST, n_tiles);
   }
 
   // score phase: thread = key (warp & 1) * 32 + lane, rows rg + 4 k
@@ -255,8 +257,17 @@ __global__ void __launch_bounds__(256, (DecodeCfg<HD, RB>::MIN_BLOCKS))
       }
     }
     __syncthreads();  // stage s and the P buffer are free again
-    if (tid == 0 && ok && t + ST < n_tiles) issue(t + ST);
+    if (tid == 0 && ok && t + ST < n_tiles) {
+      issue(t + ST);
+      issued = t + ST + 1;
+    }
   }
+  // leave no copy in flight into shared memory (the stages are reused below,
+  // and a bounded wait may have given up before they were consumed)
+  if (tid == 0)
+    for (int t = max(0, issued - ST); t < issued; ++t)
+      (void)mbar_wait_drain(smem_u32(&bar_full[t % ST]), (t / ST) & 1, p.timeout_ns);
+  __syncthreads();
 
   // this split's state; with key subsets, their sums are added first (the
   // subsets of a row share its max and rescale factors, so their sums add)

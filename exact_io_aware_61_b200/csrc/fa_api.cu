@@ -22,8 +22,7 @@
 #include "fwd2_sm100.cuh"
 #include "fwd_f32.cuh"
 #include "bwd_sm100.cuh"
-#include "bwd_dkdv_sm100.cuh"
-#include "bwd_dq_sm100.cuh"
+#include "bwd2_sm100.cuh"
 #include "decode_sm100.cuh"
 
 namespace {
@@ -101,10 +100,8 @@ int prepare_kernels(int dev) {
   set_decode_attributes<64>(set);
   set_decode_attributes<128>(set);
   set_decode_attributes<256>(set);
-  set(reinterpret_cast<const void*>(&fa::fa_bwd_dkdv_kernel<64>), fa::BwdKVCfg<64>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_bwd_dkdv_kernel<128>), fa::BwdKVCfg<128>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_bwd_dq_kernel<64>), fa::BwdQCfg<64>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_bwd_dq_kernel<128>), fa::BwdQCfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64>), fa::Bwd2Cfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128>), fa::Bwd2Cfg<128>::SMEM_BYTES);
   if (e != cudaSuccess) return FA_ERR_CUDA;
   done[dev] = true;
   return FA_OK;
@@ -263,9 +260,9 @@ int launch_fwd_f32(const void* q, const void* k, const void* v, void* o, float* 
 size_t padded_rows(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 
 // How many CTAs share the query heads of one (KV head, 128-key tile) in the
-// dK/dV kernel: 1 unless B * Hkv * (key tiles) is below 592 (4 CTAs per SM of
-// a 148-SM part), then the smallest divisor of the group size that reaches
-// it, or the group size. A pure function of the shape, so the workspace size
+// backward: 1 unless B * Hkv * (key tiles) is below 592 (4 CTAs per SM of a
+// 148-SM part), then the smallest divisor of the group size that reaches it,
+// or the group size. A pure function of the shape, so the workspace size
 // does not depend on the device.
 int bwd_head_split(int B, int Hq, int Hkv, int N) {
   const long long ctas = static_cast<long long>(B) * Hkv * static_cast<long long>(padded_rows(N) / 128);
@@ -275,12 +272,13 @@ int bwd_head_split(int B, int Hq, int Hkv, int N) {
   return g;
 }
 
-// Workspace carve-up, all f32: D [B*Hq][Npad], LSE*log2(e) [B*Hq][Npad];
-// when the dK/dV kernel splits a group's heads over CTAs, also dK and dV
-// accumulators [B*Hkv][N][d].
+// Workspace carve-up, all f32: D [B*Hq][Npad], LSE*log2(e) [B*Hq][Npad],
+// dQ accumulator [B*Hq][N][d]; when the backward splits a group's heads over
+// CTAs, also dK and dV accumulators [B*Hkv][N][d].
 struct BwdWorkspace {
   float* delta;
   float* lse2;
+  float* dq_acc;
   float* dk_acc;  // null without a split
   float* dv_acc;
 };
@@ -288,7 +286,7 @@ struct BwdWorkspace {
 size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   const size_t rows_q = static_cast<size_t>(B) * Hq;
   const size_t kv_acc = bwd_head_split(B, Hq, Hkv, N) > 1 ? 2 * static_cast<size_t>(B) * Hkv * N * d : 0;
-  return sizeof(float) * (2 * rows_q * padded_rows(N) + kv_acc);
+  return sizeof(float) * (2 * rows_q * padded_rows(N) + rows_q * static_cast<size_t>(N) * d + kv_acc);
 }
 
 BwdWorkspace carve(void* ws, int B, int Hq, int Hkv, int N, int d) {
@@ -298,8 +296,9 @@ BwdWorkspace carve(void* ws, int B, int Hq, int Hkv, int N, int d) {
   BwdWorkspace w;
   w.delta = static_cast<float*>(ws);
   w.lse2 = w.delta + rows_q * npad;
+  w.dq_acc = w.lse2 + rows_q * npad;
   const bool split = bwd_head_split(B, Hq, Hkv, N) > 1;
-  w.dk_acc = split ? w.lse2 + rows_q * npad : nullptr;
+  w.dk_acc = split ? w.dq_acc + rows_q * static_cast<size_t>(N) * d : nullptr;
   w.dv_acc = split ? w.dk_acc + kv_elems : nullptr;
   return w;
 }
@@ -310,40 +309,40 @@ unsigned grid_stride_blocks(size_t n4) {
 }
 
 // Everything the backward's launches need, built (tensor maps encoded, grid
-// sizes checked) before the first of them is queued, so that every error
-// return of a backward entry point comes before any kernel runs.
+// sizes and the main kernel's register count checked) before the first of
+// them is queued, so that every error return of a backward entry point other
+// than a failed launch comes before any kernel runs.
 struct BwdPlan {
-  int d;
   cudaStream_t stream;
   BwdWorkspace w;
-  size_t kv_elems;
+  size_t kv_elems, q_elems;
   int split;
-  // prep
   fa::BwdPrepParams pp;
   unsigned prep_blocks;
-  // dK/dV
-  CUtensorMap kv_mq, kv_mdo;
-  fa::BwdKVParams kp;
-  unsigned kv_blocks;
-  // dQ
-  CUtensorMap q_mk, q_mv;
-  fa::BwdQParams qp;
-  unsigned q_blocks;
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  fa::Bwd2Params mp;
+  unsigned main_blocks;
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
 };
 
-// stages: bit 0 prep, bit 1 dK/dV, bit 2 dQ. Pointers a stage does not use may be null.
+// stages: bit 0 prep, bit 1 main, bit 2 dQ conversion. Pointers a stage does not use may be null.
+template <int HD>
 int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const void* v, const void* o,
              const float* lse, const void* dO, void* dq, void* dk, void* dv, void* ws, int B, int Hq, int Hkv,
-             int N, int d, float scale, int causal, cudaStream_t stream) {
-  pl->d = d;
+             int N, float scale, int causal, cudaStream_t stream) {
+  using C = fa::Bwd2Cfg<HD>;
   pl->stream = stream;
-  pl->w = carve(ws, B, Hq, Hkv, N, d);
-  pl->kv_elems = static_cast<size_t>(B) * Hkv * static_cast<size_t>(N) * d;
+  pl->w = carve(ws, B, Hq, Hkv, N, HD);
+  pl->kv_elems = static_cast<size_t>(B) * Hkv * static_cast<size_t>(N) * HD;
+  pl->q_elems = static_cast<size_t>(B) * Hq * static_cast<size_t>(N) * HD;
   pl->split = bwd_head_split(B, Hq, Hkv, N);
+  pl->dq = static_cast<__nv_bfloat16*>(dq);
+  pl->dk = static_cast<__nv_bfloat16*>(dk);
+  pl->dv = static_cast<__nv_bfloat16*>(dv);
   const size_t npad = padded_rows(N);
   const uint64_t rows_q = static_cast<uint64_t>(B) * Hq, rows_kv = static_cast<uint64_t>(B) * Hkv;
-  const float scale_log2 = scale * 1.4426950408889634f;
-  const unsigned long long tmo = timeout_now();
   if (stages & 1u) {
     fa::BwdPrepParams& pp = pl->pp;
     pp.o = static_cast<const __nv_bfloat16*>(o);
@@ -351,6 +350,7 @@ int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const v
     pp.lse = lse;
     pp.ws_delta = pl->w.delta;
     pp.ws_lse2 = pl->w.lse2;
+    pp.dq_acc = pl->w.dq_acc;
     pp.N = N;
     pp.Npad = static_cast<int>(npad);
     const long long blocks = static_cast<long long>(npad / 32) * B * Hq;
@@ -358,99 +358,79 @@ int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const v
     pl->prep_blocks = static_cast<unsigned>(blocks);
   }
   if (stages & 2u) {
-    int rc = make_map(&pl->kv_mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, rows_q, 64, 64);
-    if (rc == FA_OK) rc = make_map(&pl->kv_mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, rows_q, 64, 64);
+    // The kernel redistributes registers between warpgroups (setmaxnreg) on
+    // the assumption of exactly LAUNCH_REGS per thread at launch; a build
+    // with another count would wait for ever, so it is refused here.
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>)) != cudaSuccess)
+      return FA_ERR_CUDA;
+    if (attr.numRegs != C::LAUNCH_REGS) {
+      if (verbose()) std::fprintf(stderr, "fa: backward built with %d registers, expected %d\n", attr.numRegs,
+                                  C::LAUNCH_REGS);
+      return FA_ERR_UNSUPPORTED;
+    }
+    int rc = make_map(&pl->mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
+    if (rc == FA_OK) rc = make_map(&pl->mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
+    if (rc == FA_OK) rc = make_map(&pl->mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
+    if (rc == FA_OK) rc = make_map(&pl->mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
+    if (rc == FA_OK)
+      rc = make_map(&pl->mdq, pl->w.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, N, rows_q, 32, 128);
     if (rc != FA_OK) return rc;
-    fa::BwdKVParams& kp = pl->kp;
-    kp.k = static_cast<const __nv_bfloat16*>(k);
-    kp.v = static_cast<const __nv_bfloat16*>(v);
-    kp.ws_delta = pl->w.delta;
-    kp.ws_lse2 = pl->w.lse2;
-    kp.dk = static_cast<__nv_bfloat16*>(dk);
-    kp.dv = static_cast<__nv_bfloat16*>(dv);
-    kp.dk_acc = pl->w.dk_acc;
-    kp.dv_acc = pl->w.dv_acc;
-    kp.head_split = pl->split;
-    kp.BHkv = B * Hkv;
-    kp.N = N;
-    kp.Npad = static_cast<int>(npad);
-    kp.Hq = Hq;
-    kp.Hkv = Hkv;
-    kp.num_tiles = static_cast<int>(npad / 128);
-    kp.scale_log2 = scale_log2;
-    kp.scale = scale;
-    kp.causal = causal;
-    kp.timeout_ns = tmo;
-    const long long blocks = static_cast<long long>(kp.num_tiles) * B * Hkv * pl->split;
+    fa::Bwd2Params& mp = pl->mp;
+    mp.ws_delta = pl->w.delta;
+    mp.ws_lse2 = pl->w.lse2;
+    mp.dq_acc = pl->w.dq_acc;
+    mp.dk = pl->dk;
+    mp.dv = pl->dv;
+    mp.dk_acc = pl->w.dk_acc;
+    mp.dv_acc = pl->w.dv_acc;
+    mp.head_split = pl->split;
+    mp.BHkv = B * Hkv;
+    mp.N = N;
+    mp.Npad = static_cast<int>(npad);
+    mp.Hq = Hq;
+    mp.Hkv = Hkv;
+    mp.num_tiles = static_cast<int>(npad / 128);
+    mp.scale_log2 = scale * 1.4426950408889634f;
+    mp.scale = scale;
+    mp.causal = causal;
+    mp.timeout_ns = timeout_now();
+    const long long blocks = static_cast<long long>(mp.num_tiles) * B * Hkv * pl->split;
     if (blocks > INT32_MAX) return FA_ERR_INVALID;
-    pl->kv_blocks = static_cast<unsigned>(blocks);
-  }
-  if (stages & 4u) {
-    int rc = make_map(&pl->q_mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, rows_kv, 64, 64);
-    if (rc == FA_OK) rc = make_map(&pl->q_mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, rows_kv, 64, 64);
-    if (rc != FA_OK) return rc;
-    fa::BwdQParams& qp = pl->qp;
-    qp.q = static_cast<const __nv_bfloat16*>(q);
-    qp.dO = static_cast<const __nv_bfloat16*>(dO);
-    qp.ws_delta = pl->w.delta;
-    qp.ws_lse2 = pl->w.lse2;
-    qp.dq = static_cast<__nv_bfloat16*>(dq);
-    qp.N = N;
-    qp.Npad = static_cast<int>(npad);
-    qp.Hq = Hq;
-    qp.Hkv = Hkv;
-    qp.BH = B * Hq;
-    qp.num_tiles = static_cast<int>(npad / 128);
-    qp.scale_log2 = scale_log2;
-    qp.scale = scale;
-    qp.causal = causal;
-    qp.timeout_ns = tmo;
-    const long long blocks = static_cast<long long>(qp.num_tiles) * B * Hq;
-    if (blocks > INT32_MAX) return FA_ERR_INVALID;
-    pl->q_blocks = static_cast<unsigned>(blocks);
+    pl->main_blocks = static_cast<unsigned>(blocks);
   }
   return FA_OK;
-}
-
-template <int HD>
-int launch_bwd_prep(const BwdPlan& pl) {
-  fa::fa_bwd_prep_kernel<HD><<<pl.prep_blocks, 256, 0, pl.stream>>>(pl.pp);
-  return launch_status();
-}
-
-template <int HD>
-int launch_bwd_dkdv(const BwdPlan& pl) {
-  using C = fa::BwdKVCfg<HD>;
-  if (pl.split > 1) {  // zero the f32 dK and dV accumulators (contiguous)
-    fa::fa_zero_f32_kernel<<<grid_stride_blocks(pl.kv_elems / 2), 256, 0, pl.stream>>>(pl.w.dk_acc,
-                                                                                      pl.kv_elems / 2);
-    if (launch_status() != FA_OK) return FA_ERR_CUDA;
-  }
-  fa::fa_bwd_dkdv_kernel<HD><<<pl.kv_blocks, C::THREADS, C::SMEM_BYTES, pl.stream>>>(pl.kv_mq, pl.kv_mdo, pl.kp);
-  if (launch_status(reinterpret_cast<const void*>(&fa::fa_bwd_dkdv_kernel<HD>)) != FA_OK) return FA_ERR_CUDA;
-  if (pl.split > 1) {
-    const size_t n4 = pl.kv_elems / 4;
-    fa::fa_f32_to_bf16_kernel<<<grid_stride_blocks(n4), 256, 0, pl.stream>>>(pl.w.dk_acc, pl.kp.dk, n4);
-    if (launch_status() != FA_OK) return FA_ERR_CUDA;
-    fa::fa_f32_to_bf16_kernel<<<grid_stride_blocks(n4), 256, 0, pl.stream>>>(pl.w.dv_acc, pl.kp.dv, n4);
-    if (launch_status() != FA_OK) return FA_ERR_CUDA;
-  }
-  return FA_OK;
-}
-
-template <int HD>
-int launch_bwd_dq(const BwdPlan& pl) {
-  using C = fa::BwdQCfg<HD>;
-  fa::fa_bwd_dq_kernel<HD><<<pl.q_blocks, C::THREADS, C::SMEM_BYTES, pl.stream>>>(pl.q_mk, pl.q_mv, pl.qp);
-  return launch_status(reinterpret_cast<const void*>(&fa::fa_bwd_dq_kernel<HD>));
 }
 
 template <int HD>
 int launch_bwd_stages(const BwdPlan& pl, unsigned stages) {
-  int rc = FA_OK;
-  if ((stages & 1u) && (rc = launch_bwd_prep<HD>(pl)) != FA_OK) return rc;
-  if ((stages & 2u) && (rc = launch_bwd_dkdv<HD>(pl)) != FA_OK) return rc;
-  if ((stages & 4u) && (rc = launch_bwd_dq<HD>(pl)) != FA_OK) return rc;
+  using C = fa::Bwd2Cfg<HD>;
+  if (stages & 1u) {
+    fa::fa_bwd_prep_kernel<HD><<<pl.prep_blocks, 256, 0, pl.stream>>>(pl.pp);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  if (stages & 2u) {
+    if (pl.split > 1) {  // zero the f32 dK and dV accumulators (contiguous)
+      fa::fa_zero_f32_kernel<<<grid_stride_blocks(pl.kv_elems / 2), 256, 0, pl.stream>>>(pl.w.dk_acc,
+                                                                                        pl.kv_elems / 2);
+      if (launch_status() != FA_OK) return FA_ERR_CUDA;
+    }
+    fa::fa_bwd2_main_kernel<HD><<<pl.main_blocks, C::THREADS, C::SMEM_BYTES, pl.stream>>>(pl.mq, pl.mk, pl.mv,
+                                                                                          pl.mdo, pl.mdq, pl.mp);
+    if (launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>)) != FA_OK) return FA_ERR_CUDA;
+    if (pl.split > 1) {
+      const size_t n4 = pl.kv_elems / 4;
+      fa::fa_bwd_dq_kernel<<<grid_stride_blocks(n4), 256, 0, pl.stream>>>(pl.w.dk_acc, pl.dk, n4);
+      if (launch_status() != FA_OK) return FA_ERR_CUDA;
+      fa::fa_bwd_dq_kernel<<<grid_stride_blocks(n4), 256, 0, pl.stream>>>(pl.w.dv_acc, pl.dv, n4);
+      if (launch_status() != FA_OK) return FA_ERR_CUDA;
+    }
+  }
+  if (stages & 4u) {
+    const size_t n4 = pl.q_elems / 4;
+    fa::fa_bwd_dq_kernel<<<grid_stride_blocks(n4), 256, 0, pl.stream>>>(pl.w.dq_acc, pl.dq, n4);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
   return FA_OK;
 }
 
@@ -625,10 +605,17 @@ int run_bwd(unsigned stages, std::initializer_list<const void*> ptrs, const void
   int rc = check_bwd(ptrs, ws, ws_bytes, B, Hq, Hkv, N, d, scale, causal, dtype, &dev);
   if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
   BwdPlan pl;
-  if ((rc = plan_bwd(&pl, stages, q, k, v, o, lse, dO, dq, dk, dv, ws, B, Hq, Hkv, N, d, scale, causal,
-                     reinterpret_cast<cudaStream_t>(stream))) != FA_OK)
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) {
+    if ((rc = plan_bwd<64>(&pl, stages, q, k, v, o, lse, dO, dq, dk, dv, ws, B, Hq, Hkv, N, scale, causal, s)) !=
+        FA_OK)
+      return rc;
+    return launch_bwd_stages<64>(pl, stages);
+  }
+  if ((rc = plan_bwd<128>(&pl, stages, q, k, v, o, lse, dO, dq, dk, dv, ws, B, Hq, Hkv, N, scale, causal, s)) !=
+      FA_OK)
     return rc;
-  return d == 64 ? launch_bwd_stages<64>(pl, stages) : launch_bwd_stages<128>(pl, stages);
+  return launch_bwd_stages<128>(pl, stages);
 }
 
 }  // namespace
@@ -641,18 +628,17 @@ int fa_bwd_prep(const void* o, const float* lse, const void* dO, void* workspace
                  workspace_bytes, B, Hq, Hkv, N, d, 1.0f, 0, dtype, stream);
 }
 
-int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* workspace,
+int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, void* workspace,
                 size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale, int causal, int dtype,
                 fa_stream_t stream) {
   return run_bwd(2u, {q, k, v, dO, dk, dv}, q, k, v, nullptr, nullptr, dO, nullptr, dk, dv, workspace,
                  workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype, stream);
 }
 
-int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, void* workspace,
-              size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale, int causal, int dtype,
+int fa_bwd_dq(void* dq, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int dtype,
               fa_stream_t stream) {
-  return run_bwd(4u, {q, k, v, dO, dq}, q, k, v, nullptr, nullptr, dO, dq, nullptr, nullptr, workspace,
-                 workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype, stream);
+  return run_bwd(4u, {dq}, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dq, nullptr, nullptr, workspace,
+                 workspace_bytes, B, Hq, Hkv, N, d, 1.0f, 0, dtype, stream);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
@@ -714,10 +700,10 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   if ((rc = check_device(&dev)) != FA_OK) return rc;
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(dev, &scratch)) != FA_OK) return rc;
-  // Every scratch byte this problem reads is rewritten first (D and LSE by
-  // the prep kernel; the dK/dV accumulators, when the group's heads are
-  // split, by a zeroing kernel before the dK/dV kernel), so what an earlier
-  // call left in the array does not matter.
+  // Every scratch byte this problem reads is rewritten first (D, LSE and the
+  // dQ accumulator by the prep kernel; the dK/dV accumulators, when the
+  // group's heads are split, by a zeroing kernel before the main kernel), so
+  // what an earlier call left in the array does not matter.
   return run_bwd(7u, {q, k, v, o, lse, dO, dq, dk, dv}, q, k, v, o, lse, dO, dq, dk, dv, scratch,
                  kNoAllocScratchBytes, B, Hq, Hkv, N, d, scale, causal, dtype, stream);
 }

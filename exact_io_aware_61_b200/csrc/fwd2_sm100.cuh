@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(384, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q, bar_kfull[KST], bar_kempty[KST], bar_vfull[VST], bar_vempty[VST];
-  __shared__ uint64_t bar_sfull[2], bar_pfull[2], bar_odone[2];
+  __shared__ uint64_t bar_sfull[2], bar_pfull[2], bar_odone[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(smem_u32(&bar_pfull[t]), 128);
       mbar_init(smem_u32(&bar_odone[t]), 1);
     }
+    mbar_init(smem_u32(&bar_drain), 1);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -193,6 +194,7 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * (C::BM * 128), &tm_q, smem_u32(&bar_q), c * 64,
                       q0 + t * C::BM, bh);
       // order K(0), K(1), V(0), K(2), V(1), ...: K one tile ahead of V
+      int k_issued = 0, v_issued = 0;
       for (int i = 0; i <= n_max; ++i) {
         if (i < n_max) {
           const int s = i % KST;
@@ -201,6 +203,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < KCH; ++c)
             tma_load_3d(sK + s * C::KV_BYTES + c * (C::BN * 128), &tm_k, smem_u32(&bar_kfull[s]), c * 64,
                         i * C::BN, bh_kv);
+          k_issued = i + 1;
         }
         if (i >= 1) {
           const int j = i - 1, s = j % VST;
@@ -209,8 +212,16 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < KCH; ++c)
             tma_load_3d(sV + s * C::KV_BYTES + c * (C::BN * 128), &tm_v, smem_u32(&bar_vfull[s]), c * 64,
                         j * C::BN, bh_kv);
+          v_issued = j + 1;
         }
       }
+      // leave no copy in flight into shared memory (a bounded wait elsewhere
+      // may have given up before these stages were consumed)
+      (void)mbar_wait_drain(smem_u32(&bar_q), 0, p.timeout_ns);
+      for (int i = max(0, k_issued - KST); i < k_issued; ++i)
+        (void)mbar_wait_drain(smem_u32(&bar_kfull[i % KST]), (i / KST) & 1, p.timeout_ns);
+      for (int j = max(0, v_issued - VST); j < v_issued; ++j)
+        (void)mbar_wait_drain(smem_u32(&bar_vfull[j % VST]), (j / VST) & 1, p.timeout_ns);
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
@@ -265,6 +276,9 @@ __global__ void __launch_bounds__(384, 1)
         mma_commit(smem_u32(&bar_vempty[s]));
         if (k_next_ready) mma_commit(smem_u32(&bar_kempty[(j + 1) % KST]));
       }
+      // no MMA may be in flight when tensor memory is released
+      mma_commit(smem_u32(&bar_drain));
+      (void)mbar_wait_drain(smem_u32(&bar_drain), 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------- softmax

@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(192, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q, bar_kfull[ST], bar_kempty[ST], bar_vfull[ST], bar_vempty[ST];
-  __shared__ uint64_t bar_sfull[2], bar_pfull[2], bar_odone;
+  __shared__ uint64_t bar_sfull[2], bar_pfull[2], bar_odone, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(smem_u32(&bar_pfull[s]), 128);
     }
     mbar_init(smem_u32(&bar_odone), 1);
+    mbar_init(smem_u32(&bar_drain), 1);
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -125,6 +126,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive_expect_tx(smem_u32(&bar_q), C::Q_BYTES);
       for (int c = 0; c < KCH; ++c)
         tma_load_3d(sQ + c * (C::BM * 128), &tm_q, smem_u32(&bar_q), c * 64, q0, bh);
+      int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % ST;
         const uint32_t ph = (j / ST) & 1;
@@ -133,12 +135,20 @@ __global__ void __launch_bounds__(192, 1)
         for (int c = 0; c < KCH; ++c)
           tma_load_3d(sK + s * C::KV_BYTES + c * (C::BN * 128), &tm_k, smem_u32(&bar_kfull[s]), c * 64,
                       j * C::BN, bh_kv);
+        k_issued = j + 1;
         if (!mbar_wait(smem_u32(&bar_vempty[s]), ph ^ 1, wc)) break;
         mbar_arrive_expect_tx(smem_u32(&bar_vfull[s]), C::KV_BYTES);
         for (int c = 0; c < KCH; ++c)
           tma_load_3d(sV + s * C::KV_BYTES + c * (C::BN * 128), &tm_v, smem_u32(&bar_vfull[s]), c * 64,
                       j * C::BN, bh_kv);
+        v_issued = j + 1;
       }
+      // leave no copy in flight into shared memory
+      (void)mbar_wait_drain(smem_u32(&bar_q), 0, p.timeout_ns);
+      for (int j = max(0, k_issued - ST); j < k_issued; ++j)
+        (void)mbar_wait_drain(smem_u32(&bar_kfull[j % ST]), (j / ST) & 1, p.timeout_ns);
+      for (int j = max(0, v_issued - ST); j < v_issued; ++j)
+        (void)mbar_wait_drain(smem_u32(&bar_vfull[j % ST]), (j / ST) & 1, p.timeout_ns);
     }
   } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issuer
@@ -179,6 +189,9 @@ __global__ void __launch_bounds__(192, 1)
           mma_commit(smem_u32(&bar_odone));
         }
       }
+      // no MMA may be in flight when tensor memory is released
+      mma_commit(smem_u32(&bar_drain));
+      (void)mbar_wait_drain(smem_u32(&bar_drain), 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------- softmax

@@ -102,11 +102,12 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
 /*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs: the
  * per-row term D = rowsum(dO * O) and the log2-scaled LSE, both float32 and
- * padded to a multiple of 128 rows per head: 2 * B * Hq * Npad * 4 bytes,
- * Npad = N rounded up to 128. When B * Hkv * ceil(N / 128) < 592, the dK/dV
- * kernel splits each group's query heads over several CTAs (the smallest
- * divisor s of Hq / Hkv with that product times s >= 592, else Hq / Hkv) and
- * the workspace also holds float32 dK and dV accumulators [B][Hkv][N][d].
+ * padded to a multiple of 128 rows per head, plus a float32 dQ accumulator
+ * [B][Hq][N][d]: 4 * (2 * B * Hq * Npad + B * Hq * N * d) bytes, Npad = N
+ * rounded up to 128. When B * Hkv * ceil(N / 128) < 592, the backward
+ * splits each group's query heads over several CTAs (the smallest divisor s
+ * of Hq / Hkv with that product times s >= 592, else Hq / Hkv) and the
+ * workspace also holds float32 dK and dV accumulators [B][Hkv][N][d].
  * Linear in N: nothing N x N is ever allocated. Returns 0 for invalid sizes.
  */
 FA_API size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
@@ -128,13 +129,14 @@ FA_API size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
  * dV = P^T dO, dP = dO V^T, dS = P * (dP - D), dQ = scale dS K,
  * dK = scale dS^T Q. Supports dtype FA_BF16 with d in {64, 128}; other
  * combinations return FA_ERR_UNSUPPORTED. Three kernels run in stream order:
- * D and LSE preparation, the key-side kernel (dK, dV; per 128-key tile) and
- * the query-side kernel (dQ; per 128-query tile, which recomputes S and dP a
- * second time so that dQ is accumulated on chip and written once). The
- * result is deterministic, except dk and dv when the query heads are split
- * (see fa_bwd_workspace_size): then the CTAs' f32 shares are added in the
- * order they finish, and the dK/dV stage also zeroes the accumulators
- * before, and rounds them to dk, dv after, its kernel.
+ * D and LSE preparation (and zeroing of the dQ accumulator), the main
+ * recompute kernel (one CTA per 128-key tile: dK and dV, and each dQ tile
+ * added into the f32 accumulator), and the dQ conversion; with split query
+ * heads (see fa_bwd_workspace_size) the main stage also zeroes the dK/dV
+ * accumulators before, and rounds them to dk, dv after, its kernel. dq is
+ * summed in whatever order the key tiles finish, so it can differ in the
+ * last bit from run to run; dk and dv are bit-for-bit repeatable unless the
+ * query heads are split.
  */
 FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o,
            const float* lse, const void* dO, void* dq, void* dk, void* dv,
@@ -145,33 +147,31 @@ FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o,
 /*
  * The three stages of fa_bwd as separate calls, for callers that want to
  * time or schedule them one by one. Calling them in this order on one
- * stream, with the same sizes and workspace, is exactly fa_bwd (fa_bwd_dkdv
- * and fa_bwd_dq read only what fa_bwd_prep wrote, so they may also run
- * concurrently on two streams once it has finished, unless the query heads
- * are split). Arguments mean what they mean for fa_bwd; the same checks and
- * error codes apply.
+ * stream, with the same sizes and workspace, is exactly fa_bwd. Arguments
+ * mean what they mean for fa_bwd; the same checks and error codes apply.
  *
  * fa_bwd_prep -- writes D = rowsum(dO * O) and LSE * log2(e) into the
  *   workspace (128-row padded per head; padding rows get D = 0 and an
- *   infinite LSE, i.e. zero weight). Reads o, lse, dO.
- * fa_bwd_dkdv -- per 128-key tile of each KV head, rebuilds P^T and dS^T
- *   from Q, K, V, dO and the workspace rows and writes dk, dv (through f32
- *   accumulators in the workspace when the query heads are split).
- * fa_bwd_dq -- per 128-query tile of each query head, rebuilds P and dS and
- *   writes dq.
+ *   infinite LSE, i.e. zero weight) and zeroes the f32 dQ accumulator.
+ *   Reads o, lse, dO.
+ * fa_bwd_main -- the recompute kernel: per 128-key tile of each KV head it
+ *   rebuilds P from Q, K and the padded LSE, and forms dV, dP, dS, dK (written
+ *   to dk, dv, through f32 accumulators when the query heads are split) and
+ *   adds each dQ tile into the accumulator. Needs fa_bwd_prep to have run on
+ *   the same workspace.
+ * fa_bwd_dq -- converts the f32 dQ accumulator to dq (bf16).
  */
 FA_API int fa_bwd_prep(const void* o, const float* lse, const void* dO,
                 void* workspace, size_t workspace_bytes,
                 int B, int Hq, int Hkv, int N, int d, int dtype,
                 fa_stream_t stream);
-FA_API int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
+FA_API int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO,
                 void* dk, void* dv, void* workspace, size_t workspace_bytes,
                 int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                 int dtype, fa_stream_t stream);
-FA_API int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
-              void* dq, void* workspace, size_t workspace_bytes,
-              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
-              int dtype, fa_stream_t stream);
+FA_API int fa_bwd_dq(void* dq, void* workspace, size_t workspace_bytes,
+              int B, int Hq, int Hkv, int N, int d, int dtype,
+              fa_stream_t stream);
 
 /*
  * fa_bwd_noalloc -- fa_bwd for callers that cannot allocate device memory.
@@ -194,7 +194,8 @@ FA_API int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO
  * device, with that device current) and keeps it for the life of the
  * process; make that first call before any stream capture, and do not reset
  * the device afterwards. All calls share the one array: the call rewrites
- * every scratch byte it reads before reading it, but two calls whose kernels
+ * every scratch byte it reads before reading it (it zeroes the dQ
+ * accumulator itself), but two calls whose kernels
  * overlap on the GPU (different streams, no ordering between them) race on
  * it and give wrong results. Order such calls on one stream.
  */

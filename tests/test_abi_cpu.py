@@ -57,21 +57,21 @@ def _head_split(B, Hq, Hkv, N):
 
 
 def test_workspace_formula(lib):
-    # D and log2-scaled LSE padded to 128 rows per head
+    # D and log2-scaled LSE padded to 128 rows per head, plus an f32 dQ accumulator
     B, Hq, Hkv, N, d = 2, 16, 16, 4096, 128
     assert _head_split(B, Hq, Hkv, N) == 1
-    assert fa.fa_bwd_workspace_size(B, Hq, Hkv, N, d) == 4 * (2 * B * Hq * 4096)
+    assert fa.fa_bwd_workspace_size(B, Hq, Hkv, N, d) == 4 * (2 * B * Hq * 4096 + B * Hq * N * d)
     # few CTAs (1 x 2 KV heads x 2 key tiles): the group of 2 is split, and f32
     # dK/dV accumulators are added
     assert _head_split(1, 4, 2, 129) == 2
-    assert fa.fa_bwd_workspace_size(1, 4, 2, 129, 64) == 4 * (2 * 4 * 256 + 2 * 2 * 129 * 64)
+    assert fa.fa_bwd_workspace_size(1, 4, 2, 129, 64) == 4 * (2 * 4 * 256 + 4 * 129 * 64 + 2 * 2 * 129 * 64)
     # the split rule on a few shapes: MQA at 16k tokens, GQA at 16k (no split)
     assert _head_split(1, 32, 1, 16384) == 8
     assert _head_split(1, 32, 8, 16384) == 1
     for shape in ((1, 32, 1, 16384, 128), (1, 32, 8, 16384, 128), (1, 8, 2, 4096, 128), (3, 6, 3, 700, 64)):
         B, Hq, Hkv, N, d = shape
         kv = 2 * B * Hkv * N * d if _head_split(B, Hq, Hkv, N) > 1 else 0
-        want = 4 * (2 * B * Hq * ((N + 127) // 128 * 128) + kv)
+        want = 4 * (2 * B * Hq * ((N + 127) // 128 * 128) + B * Hq * N * d + kv)
         assert fa.fa_bwd_workspace_size(*shape) == want, shape
     assert fa.fa_bwd_workspace_size(1, 3, 2, 64, 64) == 0  # Hq not a multiple of Hkv
     # linear in N: nothing N x N

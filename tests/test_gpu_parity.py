@@ -336,6 +336,40 @@ def test_bwd_gqa_causal_b1_h32_kv8_n16384_d128(fa):
     assert worst <= GRAD_TOL, worst
 
 
+def test_pair_shards_on_one_gpu_match_the_single_call(fa):
+    """The (batch, KV head) partition used across GPUs, run on one GPU: three
+    emulated ranks each call fa_fwd and fa_bwd on views of their slice of the
+    inputs and outputs. O and LSE equal the single call's bit for bit; dQ, dK
+    and dV (f32 shares added in the order CTAs finish) agree to one bf16
+    rounding step."""
+    from exact_io_aware_61_b200.shard import kv_view, pair_range, q_view
+
+    B, Hq, Hkv, N, d = 2, 8, 4, 1000, 128
+    scale = d ** -0.5
+    inp = INP.make_inputs(B, Hq, Hkv, N, d, "bf16", seed=404, grad=True)
+    q, k, v, do = (_to_dev(inp[n]) for n in ("q", "k", "v", "do"))
+    o_full, lse_full = fa.forward(q, k, v, causal=True, scale=scale)
+    ref = fa.backward(q, k, v, o_full, lse_full, do, causal=True, scale=scale)
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((B, Hq, N), float("nan"), device="cuda")
+    grads = [torch.full_like(t, float("nan")) for t in ref]
+    world = 3
+    for rank in range(world):
+        s = pair_range(B, Hq, Hkv, rank, world)
+        qv, dov, ov, lv, dqv = (q_view(t, s) for t in (q, do, o, lse, grads[0]))
+        kvv, vvv, dkv, dvv = (kv_view(t, s) for t in (k, v, grads[1], grads[2]))
+        fa.fa_fwd(qv, kvv, vvv, ov, lv, True, scale)
+        ws = torch.empty(max(fa.fa_bwd_workspace_size(*s.local_shape(), N, d), 16), dtype=torch.uint8,
+                         device="cuda")
+        fa.fa_bwd(qv, kvv, vvv, ov, lv, dov, dqv, dkv, dvv, ws, True, scale)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.FA_OK
+    assert torch.equal(o, o_full) and torch.equal(lse, lse_full)
+    for got, want in zip(grads, ref):
+        diff = (got.float() - want.float()).abs()
+        assert bool(torch.all(diff <= 2.0 ** -7 * want.float().abs() + 1e-30))
+
+
 # ------------------------------------------------------- KV-cache forward
 
 KVCACHE_SHAPES = [  # (B, Hq, Hkv, Nq, Nk, d)

@@ -6,10 +6,10 @@ fa_bwd_noalloc keeps its scratch in a fixed array inside the library. This
 test calls it through the C ABI twice in a row (the second call finds the
 first call's leftovers in the shared array) and checks each result against
 fa_bwd with a caller-allocated workspace: bit for bit where the backward is
-deterministic (dQ always; dK and dV when a KV head's query heads are not
-split over CTAs), within one bf16 rounding step where split CTAs add their
-f32 shares in whatever order they finish, and against the fp64 oracle at the
-gradient tolerance the other tests use. Outputs are canary-guarded. It lives
+deterministic (dK and dV when a KV head's query heads are not split over
+CTAs), within one bf16 rounding step where f32 shares are added in whatever
+order CTAs finish (dQ always; dK and dV with split heads), and against the
+fp64 oracle at the gradient tolerance the other tests use. Outputs are canary-guarded. It lives
 in its own file, collected last, and passes both alone in a fresh process and
 after the rest of the suite.
 """
@@ -82,7 +82,7 @@ def test_noalloc_matches_fa_bwd_twice(fa, shape, causal):
         for name, g, r, o64 in zip(("dq", "dk", "dv"), guards, ref, (oq, ok_, ov)):
             got = g.t
             assert torch.isfinite(got).all(), name
-            if name == "dq" or split == 1:
+            if name != "dq" and split == 1:
                 assert torch.equal(got, r), (name, seed, "differs from fa_bwd")
             else:
                 diff = (got.float() - r.float()).abs()
