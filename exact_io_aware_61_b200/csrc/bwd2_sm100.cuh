@@ -20,22 +20,23 @@
 // accumulators that a conversion kernel rounds afterwards. Roles (16 warps):
 //   warps 0-7   two compute warpgroups; warpgroup h owns query columns
 //               [64h, 64h + 64): P^T = exp2(S^T * scale * log2 e - LSE2) ->
-//               bf16 over its own S^T columns in TMEM, then
-//               dS^T = P^T (dP^T - D) scale (bf16) -> TMEM, over the other
-//               half of those S^T columns (A operand of dK), and -> shared
-//               memory (operand of dQ)
+//               bf16 over its own S^T columns in TMEM (A operand of dV),
+//               then dS^T = P^T (dP^T - D) scale (bf16) -> shared memory,
+//               where it is the A operand of dK (read as keys x queries) and
+//               of dQ (read as queries x keys)
 //   warps 8-11  dQ drain: the dQ tile leaves TMEM at once, then is added to
 //               the f32 accumulator with TMA tensor reduce-adds
 //   warp 12     TMA producer (K, V once; Q, LSE2, D double-buffered; dO)
 //   warp 13     TMEM allocator and MMA issuer; warps 14, 15 idle
 // MMA order per step t (query tile):
-//   dP^T(t) [once dQ(t-1) left TMEM], dV += P^T dO, dK += dS^T Q,
-//   dQ(t) [into the dP^T columns], then S^T(t+1) at once, so the compute
-//   warpgroups start on step t+1 while the drain empties dQ(t).
-// Operand forms: an MMA whose A operand is in TMEM runs at the full rate,
-// one with both operands in shared memory is markedly slower, so dV and dK
-// take their A operand (P^T, dS^T) from TMEM.
+//   dP^T(t) [once dQ(t-1) left TMEM], dV += P^T dO, S^T(t+1) [over P^T(t),
+//   which dV(t) has read], dK += dS^T Q, dQ(t) [into the dP^T columns]: the
+//   next step's scores are ready while the compute warpgroups form dS^T(t),
+//   and the drain empties dQ(t) while they work on step t+1.
 // TMEM: S^T / P^T at 0, dP^T / dQ at 128, dV at 256, dK at 256 + d.
+// Every MMA runs 128 x 128 (or 128 x d) per instruction, the size at which
+// operands in shared memory and in tensor memory both keep the tensor core
+// at its full rate.
 #pragma once
 
 #include <cuda.h>
@@ -263,26 +264,28 @@ __global__ void __launch_bounds__(512, 1)
                       sdesc_sw128(dob + kk * 2048, 16384, 1024), id_kmn,
                       (t > 0 || kk > 0));
         mma_commit(smem_u32(&bar_doempty[sd]));
-        // dK += dS^T Q ; dQ = dS K
+        // S^T(t+1) may overwrite P^T(t) now (MMAs run in issue order, dV(t)
+        // first); dS^T(t) lives in shared memory, so the next step's scores
+        // are computed while the compute warpgroups form dS^T(t)
+        if (t + 1 < steps) {
+          if (!mbar_wait(smem_u32(&bar_qfull[(t + 1) % QST]), ((t + 1) / QST) & 1, wc)) break;
+          tc_fence_after();
+          issue_s(t + 1);
+        }
+        // dK += dS^T Q (A = dS^T in shared memory, keys x queries, K-major);
+        // dQ = dS K (the same buffer read as dS, queries x keys, M-major)
         if (!mbar_wait(smem_u32(&bar_dsfull), t & 1, wc)) break;
         tc_fence_after();
-        // (dS^T from TMEM: queries 64h + 32 .. of warpgroup h's columns)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + C::T_DK, tmem + C::T_S + (kk >> 2) * 64 + 32 + (kk & 3) * 8,
+          mma_bf16_ss(tmem + C::T_DK, sdesc_sw128(sDS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                       sdesc_sw128(qst + kk * 2048, 16384, 1024), id_kmn, (t > 0 || kk > 0));
-        // dQ = dS K (M = queries, N = d)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ss(tmem + C::T_DP, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
                       sdesc_sw128(sK + kk * 2048, 16384, 1024), id_mnmn, kk > 0);
         mma_commit(smem_u32(&bar_qempty[sq]));
         mma_commit(smem_u32(&bar_dqfull));
-        if (t + 1 < steps) {
-          if (!mbar_wait(smem_u32(&bar_qfull[(t + 1) % QST]), ((t + 1) / QST) & 1, wc)) break;
-          tc_fence_after();
-          issue_s(t + 1);
-        }
       }
       // bar_final completes once every MMA issued above has completed (on
       // the normal path and after a bounded wait gave up alike); no MMA may
@@ -318,33 +321,36 @@ __global__ void __launch_bounds__(512, 1)
       if (!warp_wait(smem_u32(&bar_qfull[sq]), (t / QST) & 1, wc)) { ok = false; break; }
       if (!warp_wait(smem_u32(&bar_sfull), t & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      // ---- P^T = exp2(S^T * scale * log2 e - LSE2), masked
+      // ---- P^T = exp2(S^T * scale * log2 e - LSE2), masked; kept in
+      // registers too, since S^T(t+1) overwrites these columns once dV(t) has
+      // read them
       const bool diag = p.causal && (q0 == k0);
-      {
-        uint32_t rr[2][32];
+      uint32_t pk[32];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          tmem_ld32(tmem + lane_base + C::T_S + cb + 32 * u, rr[u]);
-          uint32_t pk[16];
+      for (int u = 0; u < 2; ++u) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_base + C::T_S + cb + 32 * u, rr);
 #pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            const float4 L = l4[u * 8 + x];
-            const int qa = cb + u * 32 + 4 * x;  // query column of element 0
-            float pv[4];
-            pv[0] = ex2_approx(fmaf(__uint_as_float(rr[u][4 * x]), p.scale_log2, -L.x));
-            pv[1] = ex2_approx(fmaf(__uint_as_float(rr[u][4 * x + 1]), p.scale_log2, -L.y));
-            pv[2] = ex2_approx(fmaf(__uint_as_float(rr[u][4 * x + 2]), p.scale_log2, -L.z));
-            pv[3] = ex2_approx(fmaf(__uint_as_float(rr[u][4 * x + 3]), p.scale_log2, -L.w));
-            if (diag) {
+        for (int x = 0; x < 8; ++x) {
+          const float4 L = l4[u * 8 + x];
+          const int qa = cb + u * 32 + 4 * x;  // query column of element 0
+          float pv[4];
+          pv[0] = ex2_approx(fmaf(__uint_as_float(rr[4 * x]), p.scale_log2, -L.x));
+          pv[1] = ex2_approx(fmaf(__uint_as_float(rr[4 * x + 1]), p.scale_log2, -L.y));
+          pv[2] = ex2_approx(fmaf(__uint_as_float(rr[4 * x + 2]), p.scale_log2, -L.z));
+          pv[3] = ex2_approx(fmaf(__uint_as_float(rr[4 * x + 3]), p.scale_log2, -L.w));
+          if (diag) {
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (q0 + qa + e < key) pv[e] = 0.f;
-            }
-            pk[2 * x] = key_live ? pack_bf16x2(pv[0], pv[1]) : 0u;
-            pk[2 * x + 1] = key_live ? pack_bf16x2(pv[2], pv[3]) : 0u;
+            for (int e = 0; e < 4; ++e)
+              if (q0 + qa + e < key) pv[e] = 0.f;
           }
-          tmem_st16(tmem + lane_base + C::T_S + cb + u * 16, pk);
+          pk[u * 16 + 2 * x] = key_live ? pack_bf16x2(pv[0], pv[1]) : 0u;
+          pk[u * 16 + 2 * x + 1] = key_live ? pack_bf16x2(pv[2], pv[3]) : 0u;
         }
+        uint32_t half_pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) half_pk[i] = pk[u * 16 + i];
+        tmem_st16(tmem + lane_base + C::T_S + cb + u * 16, half_pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -355,23 +361,20 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_after();
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        uint32_t r[32], pr[16];
-        tmem_ld32_async(tmem + lane_base + C::T_DP + cb + u * 32, r);
-        tmem_ld16_async(tmem + lane_base + C::T_S + cb + u * 16, pr);
-        tmem_wait_ld32(r);
-        tmem_tie16(pr);
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + C::T_DP + cb + u * 32, r);
         uint32_t w[16];
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
           const float4 Dv = d4[u * 8 + x];
-          const float e0 = bf16_lo(pr[2 * x]) * (__uint_as_float(r[4 * x]) - Dv.x) * p.scale;
-          const float e1 = bf16_hi(pr[2 * x]) * (__uint_as_float(r[4 * x + 1]) - Dv.y) * p.scale;
-          const float e2 = bf16_lo(pr[2 * x + 1]) * (__uint_as_float(r[4 * x + 2]) - Dv.z) * p.scale;
-          const float e3 = bf16_hi(pr[2 * x + 1]) * (__uint_as_float(r[4 * x + 3]) - Dv.w) * p.scale;
+          const uint32_t p01 = pk[u * 16 + 2 * x], p23 = pk[u * 16 + 2 * x + 1];
+          const float e0 = bf16_lo(p01) * (__uint_as_float(r[4 * x]) - Dv.x) * p.scale;
+          const float e1 = bf16_hi(p01) * (__uint_as_float(r[4 * x + 1]) - Dv.y) * p.scale;
+          const float e2 = bf16_lo(p23) * (__uint_as_float(r[4 * x + 2]) - Dv.z) * p.scale;
+          const float e3 = bf16_hi(p23) * (__uint_as_float(r[4 * x + 3]) - Dv.w) * p.scale;
           w[2 * x] = pack_bf16x2(e0, e1);
           w[2 * x + 1] = pack_bf16x2(e2, e3);
         }
-        tmem_st16(tmem + lane_base + C::T_S + cb + 32 + u * 16, w);
         // 32 queries = 64 bytes = four 16-byte chunks: chunk u*4 + v, swizzled by row
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -379,7 +382,6 @@ __global__ void __launch_bounds__(512, 1)
           *reinterpret_cast<uint4*>(ds_row + chunk * 16) = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
-      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(smem_u32(&bar_dsfull));
