@@ -26,12 +26,15 @@ from ._lib import (  # noqa: F401
     fa_bwd_workspace_size,
     fa_fwd,
     fa_fwd_kvcache,
+    fa_fwd_varlen,
     fa_fwd_kvcache_workspace_size,
     fa_last_device_status,
     fa_selftest_wait_timeout,
     fa_set_wait_timeout_ns,
     forward,
+    forward_bnhd,
     forward_kvcache,
+    forward_varlen,
     load,
     status_string,
 )

@@ -22,6 +22,7 @@ FA_BF16, FA_F32 = 0, 1
 
 EXPORTED = (
     "fa_fwd",
+    "fa_fwd_varlen",
     "fa_bwd",
     "fa_bwd_prep",
     "fa_bwd_main",
@@ -60,6 +61,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
         lib.fa_fwd.restype = i
+        lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, vp]
+        lib.fa_fwd_varlen.restype = i
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp]
         lib.fa_bwd.restype = i
         lib.fa_bwd_prep.argtypes = [vp, vp, vp, vp, sz, i, i, i, i, i, i, vp]
@@ -129,6 +132,45 @@ def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
                        int(bool(causal)), _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
     if rc != FA_OK:
         raise FAError(rc, "fa_fwd")
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, max_seqlen_q: int, causal: bool, scale: float, stream=None) -> None:
+    """Call ``fa_fwd_varlen``: q [total_q, Hq, d], k/v [total_k, Hkv, d], o like q, lse [total_q, Hq] f32;
+    cu_q, cu_k int32 CUDA tensors of batch + 1 offsets."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse), ("cu_q", cu_q), ("cu_k", cu_k)):
+        _check_tensor(name, t, q.device)
+    if cu_q.dtype != torch.int32 or cu_k.dtype != torch.int32:
+        raise TypeError("cu_q and cu_k must be int32")
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    rc = load().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_q), _ptr(cu_k),
+                              cu_q.numel() - 1, int(max_seqlen_q), total_q, total_k, Hq, Hkv, d, float(scale),
+                              int(bool(causal)), _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_varlen")
+
+
+def forward_varlen(q, k, v, cu_q, cu_k, max_seqlen_q: int, causal: bool = False, scale: float | None = None,
+                   stream=None):
+    """Allocate O [total_q, Hq, d] and LSE [total_q, Hq] with torch and run ``fa_fwd_varlen``."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, max_seqlen_q, causal, scale, stream)
+    return o, lse
+
+
+def forward_bnhd(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """Forward over strided [B, N, H, d] tensors (a packed batch of B sequences of N tokens).
+
+    Returns ``(o [B, N, Hq, d], lse [B, N, Hq])``; runs ``fa_fwd_varlen`` with offsets 0, N, ..., B*N.
+    """
+    B, N, Hq, d = q.shape
+    offs = torch.arange(0, (B + 1) * N, N, dtype=torch.int32, device=q.device)
+    o, lse = forward_varlen(q.reshape(B * N, Hq, d), k.reshape(B * N, k.shape[2], d), v.reshape(B * N, v.shape[2], d),
+                            offs, offs, N, causal, scale, stream)
+    return o.view(B, N, Hq, d), lse.view(B, N, Hq)
 
 
 def fa_bwd_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:

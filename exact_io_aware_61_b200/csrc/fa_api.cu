@@ -93,6 +93,8 @@ int prepare_kernels(int dev) {
   };
   set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<64>), fa::Fwd2Cfg<64>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<128>), fa::Fwd2Cfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<64, true>), fa::Fwd2Cfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<128, true>), fa::Fwd2Cfg<128>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<256>), fa::FwdCfg<256>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<64>), fa::fwd_f32_smem_bytes<64>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<128>), fa::fwd_f32_smem_bytes<128>());
@@ -117,6 +119,22 @@ int make_map(CUtensorMap* map, const void* ptr, CUtensorMapDataType type, uint64
   const cuuint64_t dims[3] = {inner, rows, outer};
   const cuuint64_t strides[2] = {inner * elem_bytes, inner * rows * elem_bytes};
   const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = encode(map, type, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Rank-3 tiled map over a dense [d2][d1][d0] tensor with a (b0 x b1 x b2) box
+// and 128-byte swizzle; out-of-bounds reads fill zeros.
+int make_map3(CUtensorMap* map, const void* ptr, CUtensorMapDataType type, uint64_t elem_bytes, uint64_t d0,
+              uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return FA_ERR_CUDA;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * elem_bytes, d0 * d1 * elem_bytes};
+  const cuuint32_t box[3] = {b0, b1, b2};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = encode(map, type, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -235,6 +253,47 @@ int launch_fwd_bf16_2tile(const void* q, const void* k, const void* v, void* o, 
   fa::fa_fwd_bf16_2tile_kernel<HD><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv,
                                                                                                           p);
   return launch_status(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<HD>));
+}
+
+// Packed variable-length batch, d = 64 or 128: grid = tile pairs of the
+// longest sequence x sequences x heads.
+template <int HD>
+int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_q,
+                      const int* cu_k, int batch, int max_seqlen_q, int total_q, int total_k, int Hq, int Hkv,
+                      float scale, int causal, cudaStream_t stream) {
+  using C = fa::Fwd2Cfg<HD>;
+  CUtensorMap mq, mk, mv;
+  int rc = make_map3(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hq, total_q, 64, 1, 128);
+  if (rc == FA_OK) rc = make_map3(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hkv, total_k, 64, 1, 128);
+  if (rc == FA_OK) rc = make_map3(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hkv, total_k, 64, 1, 128);
+  if (rc != FA_OK) return rc;
+  fa::Fwd2Params p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = 0;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.BH = batch * Hq;
+  p.num_pairs = (max_seqlen_q + 2 * C::BM - 1) / (2 * C::BM);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.timeout_ns = timeout_now();
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.max_seqlen_q = max_seqlen_q;
+  const long long blocks = static_cast<long long>(p.num_pairs) * batch * Hq;
+  if (blocks > INT32_MAX) return FA_ERR_INVALID;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<HD, true>)) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  if (attr.numRegs != C::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;  // the register split needs exactly this
+  fa::fa_fwd_bf16_2tile_kernel<HD, true><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(
+      mq, mk, mv, p);
+  return launch_status(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<HD, true>));
 }
 
 template <int HD>
@@ -583,6 +642,33 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     case 128: return launch_fwd_f32<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
     default: return launch_fwd_f32<256>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s);
   }
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int batch, int max_seqlen_q, int total_q, int total_k, int Hq, int Hkv,
+                  int d, float scale, int causal, int dtype, fa_stream_t stream) {
+  if (batch < 0 || max_seqlen_q < 0 || total_q < 0 || total_k < 0 || Hq < 1 || Hkv < 1 || d < 1)
+    return FA_ERR_INVALID;
+  if (Hq % Hkv != 0 || (causal != 0 && causal != 1) || !std::isfinite(scale)) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if (batch == 0 || max_seqlen_q == 0 || total_q == 0) return FA_OK;
+  if (total_k < 1 || max_seqlen_q > total_q || static_cast<long long>(total_q) * Hq > INT32_MAX / 2 ||
+      static_cast<long long>(total_k) * Hkv > INT32_MAX / 2)
+    return FA_ERR_INVALID;
+  for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(lse)})
+    if (!aligned16(ptr)) return FA_ERR_INVALID;
+  for (const int* cu : {cu_seqlens_q, cu_seqlens_k})
+    if (cu == nullptr || (reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return FA_ERR_INVALID;
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != FA_OK) return rc;
+  if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_fwd_varlen<64>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q, total_q,
+                                         total_k, Hq, Hkv, scale, causal, s)
+                 : launch_fwd_varlen<128>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q,
+                                          total_q, total_k, Hq, Hkv, scale, causal, s);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {

@@ -55,7 +55,16 @@ struct Fwd2Params {
   float scale_log2;
   int causal;
   unsigned long long timeout_ns;
+  // Packed variable-length batches (the VARLEN kernel only): sequence s owns
+  // query tokens cu_q[s] .. cu_q[s+1]-1 and key tokens cu_k[s] .. cu_k[s+1]-1
+  // of Q [total_q][Hq][d] and K, V [total_k][Hkv][d]; O is laid out like Q and
+  // LSE is [total_q][Hq]. num_pairs covers max_seqlen_q.
+  const int* cu_q;
+  const int* cu_k;
+  int batch, total_q, total_k, max_seqlen_q;
 };
+
+constexpr int kStatusInvalid = 1;  // equals FA_ERR_INVALID: sequence offsets inconsistent with the sizes given
 
 // ---------------------------------------------------------------- helpers
 
@@ -101,7 +110,11 @@ FA_DEV void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
 
 // ------------------------------------------------------------------ kernel
 
-template <int HD>
+// VARLEN: packed variable-length batches (see Fwd2Params); the tensor maps
+// are then rank-3 views {d, heads, tokens} with a {64, 1, 128} box, which
+// lands in shared memory exactly like the dense {64, 128, 1} box, so only the
+// coordinates, the per-sequence lengths and the output addressing change.
+template <int HD, bool VARLEN = false>
 // 12 warps: 3 per SM sub-partition, 16384 / 96 -> 168 registers each at launch.
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_bf16_2tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -127,24 +140,58 @@ __global__ void __launch_bounds__(384, 1)
   // Work item: groups of HEAD_GROUP heads; inside a group the heaviest
   // (last) tile pairs of every head start first.
   const int bid = blockIdx.x;
-  const int per_group = C::HEAD_GROUP * p.num_pairs;
-  const int g = bid / per_group;
-  const int heads_in_group = min(C::HEAD_GROUP, p.BH - g * C::HEAD_GROUP);
-  const int r = bid - g * per_group;
-  const int pair = p.num_pairs - 1 - r / heads_in_group;
-  const int bh = g * C::HEAD_GROUP + r % heads_in_group;
-  const int b = bh / p.Hq;
-  const int hq = bh - b * p.Hq;
-  const int bh_kv = b * p.Hkv + hq / (p.Hq / p.Hkv);
+  // Dense: groups of HEAD_GROUP heads, heaviest tile pairs of every head
+  // first. Varlen: every (sequence, head) of the batch at one tile pair
+  // index, pair indices from the last (heaviest when causal) down; CTAs past
+  // their sequence's length leave at once.
+  int pair, bh, hq, bh_kv;
+  int q_len, k_len, q_tok = 0, k_tok = 0;
+  if constexpr (VARLEN) {
+    const int per_pair = p.batch * p.Hq;
+    pair = p.num_pairs - 1 - bid / per_pair;
+    const int rem = bid - (bid / per_pair) * per_pair;
+    const int sq = rem / p.Hq;
+    hq = rem - sq * p.Hq;
+    bh = sq;
+    bh_kv = hq / (p.Hq / p.Hkv);
+    q_tok = p.cu_q[sq];
+    k_tok = p.cu_k[sq];
+    q_len = p.cu_q[sq + 1] - q_tok;
+    k_len = p.cu_k[sq + 1] - k_tok;
+    const bool bad = q_tok < 0 || k_tok < 0 || q_len < 0 || k_len < q_len || q_len > p.max_seqlen_q ||
+                     q_tok + q_len > p.total_q || k_tok + k_len > p.total_k;
+    if (bad) {
+      if (threadIdx.x == 0) atomicCAS(&g_status, 0, kStatusInvalid);
+      return;
+    }
+    if (pair * 2 * C::BM >= q_len) return;  // no rows of this sequence here
+  } else {
+    const int per_group = C::HEAD_GROUP * p.num_pairs;
+    const int g = bid / per_group;
+    const int heads_in_group = min(C::HEAD_GROUP, p.BH - g * C::HEAD_GROUP);
+    const int r = bid - g * per_group;
+    pair = p.num_pairs - 1 - r / heads_in_group;
+    bh = g * C::HEAD_GROUP + r % heads_in_group;
+    const int b = bh / p.Hq;
+    hq = bh - b * p.Hq;
+    bh_kv = b * p.Hkv + hq / (p.Hq / p.Hkv);
+    q_len = k_len = p.N;
+  }
+  // query i of the (sequence's) tile sits at key position kv_off + i: the
+  // last positions when a sequence has fewer queries than keys
+  const int kv_off = k_len - q_len;
   const int q0 = pair * 2 * C::BM;
-  const int n_kv_total = (p.N + C::BN - 1) / C::BN;
+  const int n_kv_total = (k_len + C::BN - 1) / C::BN;
   int n_t[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int qs = q0 + t * C::BM;
-    n_t[t] = qs < p.N ? (p.causal ? min(qs / C::BN + 1, n_kv_total) : n_kv_total) : 0;
+    n_t[t] = qs < q_len ? (p.causal ? min((kv_off + qs + C::BM - 1) / C::BN + 1, n_kv_total) : n_kv_total) : 0;
   }
   const int n_max = max(n_t[0], n_t[1]);
+  // TMA coordinates (y, z) of query row 0 and of key row 0
+  const int qy = VARLEN ? hq : 0, qz = VARLEN ? q_tok : bh;
+  const int ky = VARLEN ? bh_kv : 0, kz = VARLEN ? k_tok : bh_kv;
 
   WaitCtl wc{&abort_flag, p.timeout_ns};
 
@@ -192,7 +239,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = 0; t < live_tiles; ++t)
         for (int c = 0; c < KCH; ++c)
           tma_load_3d(sQ + t * C::Q_TILE_BYTES + c * (C::BM * 128), &tm_q, smem_u32(&bar_q), c * 64,
-                      q0 + t * C::BM, bh);
+                      VARLEN ? qy : q0 + t * C::BM, VARLEN ? qz + q0 + t * C::BM : qz);
       // order K(0), K(1), V(0), K(2), V(1), ...: K one tile ahead of V
       int k_issued = 0, v_issued = 0;
       for (int i = 0; i <= n_max; ++i) {
@@ -202,7 +249,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(smem_u32(&bar_kfull[s]), C::KV_BYTES);
           for (int c = 0; c < KCH; ++c)
             tma_load_3d(sK + s * C::KV_BYTES + c * (C::BN * 128), &tm_k, smem_u32(&bar_kfull[s]), c * 64,
-                        i * C::BN, bh_kv);
+                        VARLEN ? ky : i * C::BN, VARLEN ? kz + i * C::BN : kz);
           k_issued = i + 1;
         }
         if (i >= 1) {
@@ -211,7 +258,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(smem_u32(&bar_vfull[s]), C::KV_BYTES);
           for (int c = 0; c < KCH; ++c)
             tma_load_3d(sV + s * C::KV_BYTES + c * (C::BN * 128), &tm_v, smem_u32(&bar_vfull[s]), c * 64,
-                        j * C::BN, bh_kv);
+                        VARLEN ? ky : j * C::BN, VARLEN ? kz + j * C::BN : kz);
           v_issued = j + 1;
         }
       }
@@ -299,8 +346,8 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t sr[128];
       tmem_ld128(s_addr, sr);
       const int key0 = j * C::BN;
-      if ((p.causal && key0 + C::BN > q0 + t * C::BM) || key0 + C::BN > p.N) {
-        const int lim = min(p.causal ? row + 1 : p.N, p.N) - key0;
+      if ((p.causal && key0 + C::BN > kv_off + q0 + t * C::BM) || key0 + C::BN > k_len) {
+        const int lim = min(p.causal ? kv_off + row + 1 : k_len, k_len) - key0;
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
@@ -380,8 +427,10 @@ __global__ void __launch_bounds__(384, 1)
     if (n > 0 && ok && warp_wait(smem_u32(&bar_odone[t]), (n - 1) & 1, wc)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const bool live = row < p.N;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (live ? row : 0)) * HD;
+      const bool live = row < q_len;
+      const size_t o_index = VARLEN ? static_cast<size_t>(q_tok + (live ? row : 0)) * p.Hq + hq
+                                    : static_cast<size_t>(bh) * p.N + (live ? row : 0);
+      __nv_bfloat16* orow = p.o + o_index * HD;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t orr[32];
@@ -397,7 +446,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 4; ++i) dst[i] = w[i];
         }
       }
-      if (live) p.lse[static_cast<size_t>(bh) * p.N + row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+      if (live) p.lse[o_index] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
     }
   }
 

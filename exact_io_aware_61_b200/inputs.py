@@ -75,3 +75,22 @@ def workload_inputs(w: Workload, seed: int = 0) -> dict:
 def as_f64(t: torch.Tensor):
     """Exact float64 numpy copy of a CPU or CUDA tensor (bf16 and f32 upcast exactly)."""
     return t.detach().to("cpu", torch.float64).numpy()
+
+
+def make_varlen_inputs(lens_q, lens_k, Hq: int, Hkv: int, d: int, dtype: str = "bf16", seed: int = 0):
+    """A packed batch of sequences: ``q [sum(lens_q), Hq, d]``, ``k, v [sum(lens_k), Hkv, d]`` (CPU) and
+    the int32 offsets ``cu_q``, ``cu_k`` (batch + 1 entries from 0). Same recipe as :func:`make_inputs`."""
+    if len(lens_q) != len(lens_k):
+        raise ValueError("one query length and one key length per sequence")
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    tq, tk = int(sum(lens_q)), int(sum(lens_k))
+    out = {
+        "q": torch.randn((tq, Hq, d), generator=g, dtype=torch.float32),
+        "k": torch.randn((tk, Hkv, d), generator=g, dtype=torch.float32),
+        "v": torch.randn((tk, Hkv, d), generator=g, dtype=torch.float32),
+    }
+    if dtype == "bf16":
+        out = {name: t.to(torch.bfloat16) for name, t in out.items()}
+    cu = lambda lens: torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32)
+    out["cu_q"], out["cu_k"] = cu(lens_q), cu(lens_k)
+    return out

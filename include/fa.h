@@ -100,6 +100,42 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
            int dtype, fa_stream_t stream);
 
 /*
+ * fa_fwd_varlen -- forward pass over a packed batch of sequences of
+ * different lengths, or over strided "BNHD" tensors.
+ *
+ *   q [total_q][Hq][d], k, v [total_k][Hkv][d]   inputs (bf16), tokens of all
+ *                                                sequences one after another
+ *   o [total_q][Hq][d]                           output (bf16)
+ *   lse [total_q][Hq]                            output, float32, natural log
+ *   cu_seqlens_q, cu_seqlens_k                   device int32 arrays of batch+1
+ *                                                non-decreasing offsets from 0:
+ *                                                sequence s owns query tokens
+ *                                                cu_seqlens_q[s] .. [s+1]-1 and
+ *                                                key tokens cu_seqlens_k[s] ..
+ *                                                [s+1]-1
+ *   max_seqlen_q                                 the longest query sequence
+ *   total_q, total_k                             tokens in q and in k, v
+ * Attention runs within each sequence and nothing crosses sequences. A
+ * sequence may have fewer queries than keys (a continued prefill, a draft):
+ * its queries are then its last positions, and with causal = 1 query i of
+ * the sequence sees its keys 0 .. (keys - queries) + i. The pages say nothing
+ * on layouts ("the softmax attention you asked for", synthetic.wiki
+ * "FlashAttention: attention's bottleneck is the wire, not the maths", "Where
+ * to be careful"); this is the plain reading. A dense [B][N][H][d] tensor is
+ * the packed layout with offsets 0, N, 2N, ..., BN, so the same call serves
+ * BNHD inputs. Supports dtype FA_BF16 with d in {64, 128}; other cases return
+ * FA_ERR_UNSUPPORTED. The offsets live on the device, so their consistency
+ * (lengths >= 0, at most max_seqlen_q queries, no more queries than keys,
+ * inside total_q and total_k) is checked by the kernel: a sequence that
+ * fails it is skipped and FA_ERR_INVALID is recorded in the device status
+ * word (fa_last_device_status). batch == 0 or total_q == 0 is a no-op.
+ */
+FA_API int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int batch,
+                  int max_seqlen_q, int total_q, int total_k, int Hq, int Hkv,
+                  int d, float scale, int causal, int dtype, fa_stream_t stream);
+
+/*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs: the
  * per-row term D = rowsum(dO * O) and the log2-scaled LSE, both float32 and
  * padded to a multiple of 128 rows per head, plus a float32 dQ accumulator
@@ -251,9 +287,11 @@ FA_API const char* fa_status_string(int status);
 
 /*
  * fa_last_device_status -- synchronises `stream`, returns the current
- * device's status word (FA_OK, or FA_ERR_TIMEOUT when some kernel gave up on
- * a bounded wait since the last call) and clears it. FA_ERR_CUDA if the
- * synchronisation itself fails.
+ * device's status word and clears it: FA_OK, or the first problem a kernel
+ * recorded since the last call -- FA_ERR_TIMEOUT (a bounded wait gave up),
+ * FA_ERR_INVALID (sequence offsets of fa_fwd_varlen inconsistent with its
+ * sizes) or FA_ERR_UNSUPPORTED (a kernel found its shared memory laid out in
+ * a way it cannot use). FA_ERR_CUDA if the synchronisation itself fails.
  */
 FA_API int fa_last_device_status(fa_stream_t stream);
 

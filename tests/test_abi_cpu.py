@@ -162,3 +162,22 @@ def test_binding_fails_loudly_without_library(tmp_path):
             _lib.load(str(tmp_path / "nope.so"))
     finally:
         _lib._handle = saved
+
+
+def test_varlen_validation_before_any_device_work(lib):
+    def call(batch=2, max_q=8, tq=16, tk=16, Hq=4, Hkv=2, d=128, scale=0.1, causal=1, dtype=0, cu=64):
+        p = ctypes.c_void_p(64)
+        c = ctypes.c_void_p(cu)
+        return lib.fa_fwd_varlen(p, p, p, p, p, c, c, batch, max_q, tq, tk, Hq, Hkv, d, scale, causal, dtype, None)
+    assert call(batch=-1) == fa.FA_ERR_INVALID
+    assert call(max_q=-1) == fa.FA_ERR_INVALID
+    assert call(Hq=3) == fa.FA_ERR_INVALID
+    assert call(causal=2) == fa.FA_ERR_INVALID
+    assert call(scale=float("nan")) == fa.FA_ERR_INVALID
+    assert call(d=256) == fa.FA_ERR_UNSUPPORTED
+    assert call(dtype=1) == fa.FA_ERR_UNSUPPORTED
+    assert call(tk=0) == fa.FA_ERR_INVALID            # queries but no keys
+    assert call(max_q=17) == fa.FA_ERR_INVALID        # longer than all the queries
+    assert call(cu=66) == fa.FA_ERR_INVALID           # misaligned offsets
+    assert call(cu=0) == fa.FA_ERR_INVALID            # no offsets
+    assert call(batch=0) == fa.FA_OK and call(tq=0, max_q=0) == fa.FA_OK  # empty
