@@ -58,6 +58,17 @@ within each sequence and nothing across sequences; the pages say nothing on
 layouts ("the softmax attention you asked for", synthetic.wiki, section "Where
 to be careful"), and the reading taken is the plain one.
 
+Queries and keys at arbitrary sequence positions (``attention_forward_positions``)
+and the merge of normalised outputs of disjoint key sets (``merge_outputs``) are
+what attention sharded over the sequence dimension computes on each device and
+combines across devices. The pages name parallelism over the sequence dimension
+(synthetic.wiki, section "Versions, and what the numbers say") and give the
+rescale rule that makes the merge exact (fanfani.net, section "A pinch of math:
+making the softmax work in pieces"), but no formula for the sharded form; the
+reading taken is the plain one: under the causal mask a key is visible to a query
+iff its position is not after the query's, and a normalised output ``O_s`` with
+its ``LSE_s`` is the softmax state ``(m = LSE_s, l = 1, o = O_s)`` of its key set.
+
 Layouts: Q, O, dO, dQ are ``[B, Hq, N, d]``; K, V, dK, dV are
 ``[B, Hkv, N, d]``; LSE and D are ``[B, Hq, N]``. All arithmetic is float64.
 """
@@ -81,6 +92,8 @@ __all__ = [
     "attention_forward_varlen",
     "partial_state",
     "merge_partial_states",
+    "attention_forward_positions",
+    "merge_outputs",
 ]
 
 
@@ -95,11 +108,12 @@ def kv_head_of(hq: int, Hq: int, Hkv: int) -> int:
     return hq // (Hq // Hkv)
 
 
-def masked_scores(q_bh, k_bh, scale: float, causal: bool, rows=None) -> np.ndarray:
+def masked_scores(q_bh, k_bh, scale: float, causal: bool, rows=None, keys=None) -> np.ndarray:
     """Scaled scores ``scale * Q K^T`` of one head, masked entries set to -inf.
 
     ``q_bh`` is ``[N, d]`` (or ``[len(rows), d]`` when ``rows`` lists the query
-    positions it holds), ``k_bh`` is ``[N, d]``. Returns ``[n_rows, N]``.
+    positions it holds), ``k_bh`` is ``[N, d]`` (at positions ``keys`` when
+    given, else ``0 .. N-1``). Returns ``[n_rows, N]``.
     """
     q_bh = _f64(q_bh)
     k_bh = _f64(k_bh)
@@ -107,7 +121,7 @@ def masked_scores(q_bh, k_bh, scale: float, causal: bool, rows=None) -> np.ndarr
     s = scale * (q_bh @ k_bh.T)
     if causal:
         qpos = np.arange(q_bh.shape[0]) if rows is None else np.asarray(rows)
-        kpos = np.arange(n_keys)
+        kpos = np.arange(n_keys) if keys is None else np.asarray(keys)
         s = np.where(kpos[None, :] <= qpos[:, None], s, -np.inf)
     return s
 
@@ -395,3 +409,48 @@ def attention_forward_varlen(q, k, v, cu_q, cu_k, scale: float, causal: bool):
             o[q0:q1, h] = p @ v[k0:k1, hk]
             lse[q0:q1, h] = _lse(m, l)
     return o, lse
+
+
+def attention_forward_positions(q, k, v, q_pos, k_pos, scale: float, causal: bool):
+    """Exact attention of queries at sequence positions ``q_pos`` against keys at ``k_pos``.
+
+    ``q`` is ``[B, Hq, Nq, d]``, ``k`` and ``v`` are ``[B, Hkv, Nk, d]``,
+    ``q_pos`` has ``Nq`` and ``k_pos`` ``Nk`` integer entries (any order). With
+    ``causal``, key ``j`` is visible to query ``i`` iff ``k_pos[j] <= q_pos[i]``.
+    A row that sees no key gets ``O = 0`` and ``LSE = -inf``. Returns
+    ``(O [B,Hq,Nq,d], LSE [B,Hq,Nq])``.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    B, Hq, Nq, _ = q.shape
+    Hkv = k.shape[1]
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    k_pos = np.asarray(k_pos, dtype=np.int64)
+    if q_pos.shape != (Nq,) or k_pos.shape != (k.shape[2],):
+        raise ValueError("one position per query row and per key row")
+    o = np.empty((B, Hq, Nq, v.shape[-1]))
+    lse = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            hk = kv_head_of(h, Hq, Hkv)
+            s = masked_scores(q[b, h], k[b, hk], scale, causal, rows=q_pos, keys=k_pos)
+            p, m, l = softmax_rows(s)
+            o[b, h] = p @ v[b, hk]
+            lse[b, h] = _lse(m, l)
+    return o, lse
+
+
+def merge_outputs(os, lses):
+    """Combine the normalised outputs of disjoint key sets into ``(O, LSE)``.
+
+    ``os`` is ``[sets, rows, d]`` and ``lses`` is ``[sets, rows]``: set ``s``
+    gave ``O_s`` and ``LSE_s`` for its keys alone. ``(O_s, LSE_s)`` is the
+    softmax state ``m = LSE_s``, ``l = 1``, ``o = O_s`` of its keys (both give
+    ``l e^m = e^LSE_s`` and ``o / l = O_s``), so :func:`merge_partial_states`
+    combines them; a set with ``LSE_s = -inf`` (no visible key) has ``l = 0``
+    and contributes nothing.
+    """
+    os, lses = _f64(os), _f64(lses)
+    finite = np.isfinite(lses)
+    return merge_partial_states(lses, finite.astype(np.float64), np.where(finite[..., None], os, 0.0))

@@ -359,7 +359,68 @@ def check_varlen_sequence_order_invariance(o):
             assert np.max(np.abs(bl[cqp[i]:cqp[i + 1]] - al[cq[s]:cq[s + 1]])) < 1e-14
 
 
+
+def check_positions_reduce_to_square_and_kvcache(o):
+    # Queries and keys at positions 0..N-1 are the square problem; queries at
+    # the last Nq of Nk positions are the (pinned) KV-cache problem.
+    q, k, v = _qkv(B=2, Hq=4, Hkv=2, N=11, d=4, seed=97)
+    for causal in (False, True):
+        ao, al = o.attention_forward(q, k, v, 0.6, causal)
+        po, pl = o.attention_forward_positions(q, k, v, np.arange(11), np.arange(11), 0.6, causal)
+        assert np.max(np.abs(po - ao)) < 1e-14 and np.max(np.abs(pl - al)) < 1e-14
+        ko, kl = o.attention_forward_kvcache(q[:, :, 7:], k, v, 0.6, causal)
+        po, pl = o.attention_forward_positions(q[:, :, 7:], k, v, np.arange(7, 11), np.arange(11), 0.6, causal)
+        assert np.max(np.abs(po - ko)) < 1e-14 and np.max(np.abs(pl - kl)) < 1e-14
+
+
+def check_positions_brute_force(o):
+    # Scalar loops over a tiny head with positions out of order, one query
+    # that sees every key and one that sees none (O = 0, LSE = -inf).
+    rng = np.random.default_rng(101)
+    q = rng.standard_normal((1, 1, 4, 3))
+    k = rng.standard_normal((1, 1, 5, 3))
+    v = rng.standard_normal((1, 1, 5, 2))
+    q_pos, k_pos = [5, -1, 2, 9], [3, 1, 4, 0, 2]
+    out, lse = o.attention_forward_positions(q, k, v, q_pos, k_pos, 0.9, True)
+    for i in range(4):
+        vis = [j for j in range(5) if k_pos[j] <= q_pos[i]]
+        if not vis:
+            assert np.all(out[0, 0, i] == 0.0) and lse[0, 0, i] == -np.inf
+            continue
+        sc = {j: 0.9 * sum(q[0, 0, i, t] * k[0, 0, j, t] for t in range(3)) for j in vis}
+        z = sum(math.exp(x) for x in sc.values())
+        assert abs(lse[0, 0, i] - math.log(z)) < 1e-13
+        for c in range(2):
+            ref = sum(math.exp(sc[j]) * v[0, 0, j, c] for j in vis) / z
+            assert abs(out[0, 0, i, c] - ref) < 1e-13
+    assert len([j for j in range(5) if k_pos[j] <= 9]) == 5
+
+
+def check_striped_shards_merge_to_full(o):
+    # Token t on shard t % W: each shard's queries against each shard's keys,
+    # merged over the key shards, give the full attention of those queries --
+    # causal blocks with a row that sees nothing included (W = 3, N = 12, GQA).
+    q, k, v = _qkv(B=1, Hq=4, Hkv=2, N=12, d=5, seed=103)
+    W = 3
+    for causal in (False, True):
+        fo, fl = o.attention_forward(q, k, v, 0.45, causal)
+        for r in range(W):
+            qp = r + W * np.arange(12 // W)
+            parts = [o.attention_forward_positions(q[:, :, r::W], k[:, :, c::W], v[:, :, c::W], qp,
+                                                   c + W * np.arange(12 // W), 0.45, causal) for c in range(W)]
+            if causal and r < W - 1:
+                assert parts[W - 1][1][0, 0, 0] == -np.inf  # query r sees no key of shard W-1 > r
+            os = np.stack([pp[0].reshape(-1, 5) for pp in parts])
+            ls = np.stack([pp[1].reshape(-1) for pp in parts])
+            mo, ml = o.merge_outputs(os, ls)
+            assert np.max(np.abs(mo - fo[:, :, r::W].reshape(-1, 5))) < 1e-13
+            assert np.max(np.abs(ml - fl[:, :, r::W].reshape(-1))) < 1e-13
+
+
 ALL_CHECKS = [
+    check_positions_reduce_to_square_and_kvcache,
+    check_positions_brute_force,
+    check_striped_shards_merge_to_full,
     check_varlen_is_each_sequence_alone,
     check_varlen_sequence_order_invariance,
     check_kvcache_is_the_last_rows_of_the_square_problem,
@@ -399,25 +460,36 @@ def _mut_sign_D(p, dp, D):  # wrong sign
     return p * (dp + D[:, None])
 
 
-def _mut_mask_strict(q_bh, k_bh, scale, causal, rows=None):  # off-by-one: j < i
+def _mut_mask_strict(q_bh, k_bh, scale, causal, rows=None, keys=None):  # off-by-one: j < i
     s = scale * (np.asarray(q_bh, float) @ np.asarray(k_bh, float).T)
     if causal:
         qpos = np.arange(s.shape[0]) if rows is None else np.asarray(rows)
-        s = np.where(np.arange(s.shape[1])[None, :] < qpos[:, None], s, -np.inf)
+        kpos = np.arange(s.shape[1]) if keys is None else np.asarray(keys)
+        s = np.where(kpos[None, :] < qpos[:, None], s, -np.inf)
     return s
 
 
-def _mut_no_scale(q_bh, k_bh, scale, causal, rows=None):  # scale dropped
-    return ORIG["masked_scores"](q_bh, k_bh, 1.0, causal, rows)
+def _mut_no_scale(q_bh, k_bh, scale, causal, rows=None, keys=None):  # scale dropped
+    return ORIG["masked_scores"](q_bh, k_bh, 1.0, causal, rows, keys)
 
 
-def _mut_transposed_keys(q_bh, k_bh, scale, causal, rows=None):  # K^T Q instead of Q K^T
+def _mut_transposed_keys(q_bh, k_bh, scale, causal, rows=None, keys=None):  # K^T Q instead of Q K^T
     s = ORIG["masked_scores"](q_bh, k_bh, scale, False, rows)
     s = s.T if s.shape[0] == s.shape[1] else s
     if causal:
         qpos = np.arange(s.shape[0]) if rows is None else np.asarray(rows)
-        s = np.where(np.arange(s.shape[1])[None, :] <= qpos[:, None], s, -np.inf)
+        kpos = np.arange(s.shape[1]) if keys is None else np.asarray(keys)
+        s = np.where(kpos[None, :] <= qpos[:, None], s, -np.inf)
     return s
+
+
+def _mut_positions_ignore_keys(q, k, v, q_pos, k_pos, scale, causal):  # key positions taken as 0..Nk-1
+    return ORIG["attention_forward_positions"](q, k, v, q_pos, np.arange(np.shape(k)[2]), scale, causal)
+
+
+def _mut_merge_outputs_plain_mean(os, lses):  # outputs averaged, LSE weights dropped
+    os, lses = np.asarray(os, float), np.asarray(lses, float)
+    return os.mean(axis=0), np.log(np.sum(np.exp(lses), axis=0))
 
 
 def _mut_softmax_no_max(s):  # max subtraction dropped
@@ -464,7 +536,8 @@ def _mut_merge_no_rescale(ms, ls, os):  # sums added without the exp(m_s - M) fa
     return np.sum(os, axis=0) / L[:, None], np.max(ms, axis=0) + np.log(L)
 
 
-ORIG = {name: getattr(ORACLE, name) for name in ("masked_scores", "softmax_rows", "score_gradient", "kv_head_of")}
+ORIG = {name: getattr(ORACLE, name) for name in ("masked_scores", "softmax_rows", "score_gradient", "kv_head_of",
+                                                 "attention_forward_positions")}
 
 MUTATIONS = [
     ("score_gradient", _mut_drop_D),
@@ -478,6 +551,8 @@ MUTATIONS = [
     ("attention_forward_kvcache", _mut_kvcache_top_left),
     ("merge_partial_states", _mut_merge_no_rescale),
     ("attention_forward_varlen", _mut_varlen_leak),
+    ("attention_forward_positions", _mut_positions_ignore_keys),
+    ("merge_outputs", _mut_merge_outputs_plain_mean),
 ]
 
 
