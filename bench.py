@@ -640,6 +640,128 @@ def run_fwd_shape(args, rank, world, local):
         "data": "synthetic: i.i.d. N(0,1), seeded"}))
 
 
+def run_seqpar(args, rank, world, local):
+    """Time the sequence-sharded causal forward (striped tokens, K/V ring, merge).
+
+    On one GPU the W ranks' work is emulated: the busiest rank's W blocks
+    (``fa_fwd_partial`` against every rank's K/V shard, all held on this GPU)
+    and its ``fa_merge_partials``, with no transfer. Under torch.distributed
+    (one rank per GPU, W = world) each rank runs ``seqpar.ring_forward`` over
+    NCCL; the time is the maximum over ranks. ``value`` is the TFLOP/s of one
+    rank's own blocks (their visible score entries x 4 d, per query head),
+    over that rank's time."""
+    import torch
+
+    import exact_io_aware_61_b200 as fa
+    from exact_io_aware_61_b200 import seqpar
+
+    B, Hq, Hkv, N, d, W = (int(x) for x in args.seqpar.split(","))
+    if world > 1 and world != W:
+        raise SystemExit("--seqpar: W must equal the number of ranks under torch.distributed")
+    if N % W:
+        raise SystemExit("--seqpar: N must be a multiple of W")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    fa.load()
+    n = N // W
+    scale = d ** -0.5
+    g = torch.Generator(device="cpu").manual_seed(SEED)
+    me = W - 1 if world == 1 else rank  # under the causal mask rank W-1 has the most visible keys
+    if world == 1:
+        q = torch.randn((B, Hq, n, d), generator=g).to(torch.bfloat16).to(dev)
+        kv = [(torch.randn((B, Hkv, n, d), generator=g).to(torch.bfloat16).to(dev),
+               torch.randn((B, Hkv, n, d), generator=g).to(torch.bfloat16).to(dev)) for _ in range(W)]
+        o_parts = torch.empty((W, B, Hq, n, d), dtype=torch.bfloat16, device=dev)
+        l_parts = torch.empty((W, B, Hq, n), dtype=torch.float32, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, n), dtype=torch.float32, device=dev)
+        sched = seqpar.ring_schedule(me, W, True)
+    else:
+        g.manual_seed(SEED + rank)
+        q, k, v = (torch.randn((B, h, n, d), generator=g).to(torch.bfloat16).to(dev) for h in (Hq, Hkv, Hkv))
+    stream = torch.cuda.current_stream(dev)
+    blk_ev = []
+
+    def run(record=False):
+        if world > 1:
+            seqpar.ring_forward(q, k, v, causal=True, scale=scale)
+            return
+        for t, (src, diag) in enumerate(sched):
+            if record:
+                e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                e[0].record(stream)
+            fa.fa_fwd_partial(q, kv[src][0], kv[src][1], o_parts[t], l_parts[t], True, scale, diag, stream)
+            if record:
+                e[1].record(stream)
+                blk_ev.append(("block", e))
+        if record:
+            e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            e[0].record(stream)
+        fa.fa_merge_partials(o_parts, l_parts, o, lse, stream)
+        if record:
+            e[1].record(stream)
+            blk_ev.append(("merge", e))
+
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    sampler = ClockSampler(physical_gpu_index(local))
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        run(record=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier(world, dev)
+    if fa.fa_last_device_status(stream) != fa.FA_OK:
+        raise RuntimeError("device status reports a timeout")
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    # visible (query, key) pairs of this rank's blocks: n(n+1)/2 on the
+    # diagonal-0 blocks, n(n-1)/2 on the diagonal -1 ones
+    pairs = sum(n * (n + 1) // 2 if diag == 0 else n * (n - 1) // 2 for _, diag in seqpar.ring_schedule(me, W, True))
+    flops = 4.0 * B * Hq * d * pairs
+    tflops = flops / ms / 1e9
+    peaks, src = load_peaks()
+    out = {
+        "metric": "sequence-sharded causal attention forward, TFLOP/s of one rank", "value": round(tflops, 2),
+        "unit": "TFLOP/s", "higher_is_better": True, "n_gpus": world, "ms_per_step": round(ms, 4),
+        "steps": args.steps, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic: i.i.d. N(0,1), seeded",
+        "config": {"workload": f"causal bf16 attention forward over N={N} tokens striped across W={W} ranks, "
+                               f"B={B} Hq={Hq} Hkv={Hkv} d={d}, {n} tokens per rank",
+                   "mode": "one GPU: rank W-1's blocks and merge, no transfer" if world == 1 else
+                           "torch.distributed ring over NCCL, max over ranks",
+                   "l2": "no flush: the per-rank working set is not larger than L2 at every W"},
+        "pct_of_peak": round(100 * tflops / peaks["bf16_tflops"], 2), "peak_note": f"{src} bf16 GEMM (burst)",
+        "clocks": clocks,
+    }
+    if world == 1:
+        blk = [a.elapsed_time(b) for kind, (a, b) in blk_ev if kind == "block"]
+        mrg = [a.elapsed_time(b) for kind, (a, b) in blk_ev if kind == "merge"]
+        mbytes = (W + 1) * B * Hq * n * (2 * d + 4)
+        merge_ms = statistics.median(mrg)
+        out["kernels"] = {
+            "fa_fwd_partial": {"ms_per_block": round(statistics.median(blk), 4),
+                               "tflops": round(flops / W / statistics.median(blk) / 1e9, 2)},
+            "fa_merge_partials": {"ms": round(merge_ms, 4), "algorithmic_bytes": mbytes,
+                                  "gbs": round(mbytes / merge_ms / 1e6, 1),
+                                  "frac_of_hbm": round(mbytes / merge_ms / 1e6 / peaks["hbm_gbs"], 4)},
+        }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return  # rank 0 alone times the oracle; the others exit without work
@@ -691,6 +813,8 @@ def main(argv=None):
                     help="B,Hq,Hkv,N,d,causal[,dtype]: time the forward alone on that shape")
     ap.add_argument("--kvcache", default=None,
                     help="B,Hq,Hkv,Nq,Nk,d: time the KV-cache (decode) forward instead of the benchmark step")
+    ap.add_argument("--seqpar", default=None,
+                    help="B,Hq,Hkv,N,d,W: time the sequence-sharded causal forward over W striped ranks")
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d of a smaller case for profiling (default: the benchmark workload)")
     args = ap.parse_args(argv)
@@ -705,7 +829,9 @@ def main(argv=None):
     if world != args.gpus:
         if world == 1 and args.gpus > 1:
             ap.error(f"--gpus {args.gpus} needs a launch with torch.distributed.run (one rank per GPU)")
-    if args.kvcache:
+    if args.seqpar:
+        run_seqpar(args, rank, world, local)
+    elif args.kvcache:
         run_kvcache(args, rank, world, local)
     elif args.fwd:
         run_fwd_shape(args, rank, world, local)

@@ -26,9 +26,11 @@ from ._lib import (  # noqa: F401
     fa_bwd_workspace_size,
     fa_fwd,
     fa_fwd_kvcache,
+    fa_fwd_partial,
     fa_fwd_varlen,
     fa_fwd_kvcache_workspace_size,
     fa_last_device_status,
+    fa_merge_partials,
     fa_selftest_wait_timeout,
     fa_set_wait_timeout_ns,
     forward,

@@ -23,6 +23,8 @@ FA_BF16, FA_F32 = 0, 1
 EXPORTED = (
     "fa_fwd",
     "fa_fwd_varlen",
+    "fa_fwd_partial",
+    "fa_merge_partials",
     "fa_bwd",
     "fa_bwd_prep",
     "fa_bwd_main",
@@ -63,6 +65,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_fwd.restype = i
         lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, vp]
         lib.fa_fwd_varlen.restype = i
+        lib.fa_fwd_partial.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
+        lib.fa_fwd_partial.restype = i
+        lib.fa_merge_partials.argtypes = [vp, vp, i, ctypes.c_longlong, vp, vp, i, i, vp]
+        lib.fa_merge_partials.restype = i
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp]
         lib.fa_bwd.restype = i
         lib.fa_bwd_prep.argtypes = [vp, vp, vp, vp, sz, i, i, i, i, i, i, vp]
@@ -148,6 +154,34 @@ def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, max_seqlen_q: int, causal: bool, 
                               int(bool(causal)), _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
     if rc != FA_OK:
         raise FAError(rc, "fa_fwd_varlen")
+
+
+def fa_fwd_partial(q, k, v, o, lse, causal: bool, scale: float, diag_offset: int, stream=None) -> None:
+    """Call ``fa_fwd_partial``: ``fa_fwd`` with query row i seeing key row j iff j <= i + diag_offset (causal)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse)):
+        _check_tensor(name, t, q.device)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    rc = load().fa_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, float(scale),
+                               int(bool(causal)), int(diag_offset), _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_partial")
+
+
+def fa_merge_partials(o_parts, lse_parts, o, lse, stream=None) -> None:
+    """Call ``fa_merge_partials``: o_parts [P, ..., d] and lse_parts [P, ...] into o [..., d] and lse [...]."""
+    for name, t in (("o_parts", o_parts), ("lse_parts", lse_parts), ("o", o), ("lse", lse)):
+        _check_tensor(name, t, o_parts.device)
+    n_parts, d = o_parts.shape[0], o_parts.shape[-1]
+    rows = o.numel() // d
+    if o_parts.numel() != n_parts * rows * d or lse_parts.numel() != n_parts * rows or lse.numel() != rows:
+        raise ValueError("o_parts, lse_parts, o and lse disagree on the number of rows")
+    if lse_parts.dtype != torch.float32 or lse.dtype != torch.float32:
+        raise TypeError("LSE tensors must be float32")
+    rc = load().fa_merge_partials(_ptr(o_parts), _ptr(lse_parts), n_parts, rows, _ptr(o), _ptr(lse), d,
+                                  _dtype_code(o_parts), ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_merge_partials")
 
 
 def forward_varlen(q, k, v, cu_q, cu_k, max_seqlen_q: int, causal: bool = False, scale: float | None = None,

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <initializer_list>
 #include <mutex>
+#include <utility>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -24,6 +25,7 @@
 #include "bwd_sm100.cuh"
 #include "bwd2_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "merge_sm100.cuh"
 
 namespace {
 
@@ -196,12 +198,12 @@ int make_qkv_maps(CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv, const void*
 
 // d = 256: one 128-row query tile per CTA (S double-buffered in TMEM).
 int launch_fwd_bf16_d256(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                         int N, float scale, int causal, cudaStream_t stream) {
+                         int N, float scale, int causal, cudaStream_t stream, int diag_shift = 0) {
   using C = fa::FwdCfg<256>;
   CUtensorMap mq, mk, mv;
   int rc = make_qkv_maps<256>(&mq, &mk, &mv, q, k, v, B, Hq, Hkv, N);
   if (rc != FA_OK) return rc;
-  fa::FwdParams p;
+  fa::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.N = N;
@@ -211,6 +213,7 @@ int launch_fwd_bf16_d256(const void* q, const void* k, const void* v, void* o, f
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal;
   p.timeout_ns = timeout_now();
+  p.diag_shift = diag_shift;
   const long long blocks = static_cast<long long>(p.num_q_tiles) * B * Hq;
   if (blocks > INT32_MAX) return FA_ERR_INVALID;
   fa::fa_fwd_bf16_kernel<256><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
@@ -220,12 +223,13 @@ int launch_fwd_bf16_d256(const void* q, const void* k, const void* v, void* o, f
 // d = 64, 128: two 128-row query tiles per CTA.
 template <int HD>
 int launch_fwd_bf16_2tile(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                          int N, float scale, int causal, cudaStream_t stream) {
+                          int N, float scale, int causal, cudaStream_t stream, int diag_shift = 0) {
   using C = fa::Fwd2Cfg<HD>;
   CUtensorMap mq, mk, mv;
   int rc = make_qkv_maps<HD>(&mq, &mk, &mv, q, k, v, B, Hq, Hkv, N);
   if (rc != FA_OK) return rc;
-  fa::Fwd2Params p;
+  fa::Fwd2Params p{};
+  p.diag_shift = diag_shift;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.N = N;
@@ -294,6 +298,25 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
   fa::fa_fwd_bf16_2tile_kernel<HD, true><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(
       mq, mk, mv, p);
   return launch_status(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<HD, true>));
+}
+
+template <int HD>
+int launch_merge(const void* o_parts, const float* lse_parts, int n_parts, long long rows, void* o, float* lse,
+                 int num_sms, cudaStream_t stream) {
+  constexpr int TPR = HD / 8;
+  const long long threads = rows * TPR;
+  const long long want = (threads + fa::MergeCfg::THREADS - 1) / fa::MergeCfg::THREADS;
+  // grid-stride over rows with exactly the blocks that are resident at once
+  // (a second, partial wave would leave its blocks a full share of rows)
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fa::fa_merge_partials_kernel<HD>,
+                                                    fa::MergeCfg::THREADS, 0) != cudaSuccess ||
+      per_sm < 1)
+    return FA_ERR_CUDA;
+  const long long blocks = std::min<long long>(want, static_cast<long long>(per_sm) * num_sms);
+  fa::fa_merge_partials_kernel<HD><<<static_cast<unsigned>(blocks), fa::MergeCfg::THREADS, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o_parts), lse_parts, n_parts, rows, static_cast<__nv_bfloat16*>(o), lse);
+  return launch_status();
 }
 
 template <int HD>
@@ -669,6 +692,61 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
                                          total_k, Hq, Hkv, scale, causal, s)
                  : launch_fwd_varlen<128>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q,
                                           total_q, total_k, Hq, Hkv, scale, causal, s);
+}
+
+int fa_fwd_partial(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                   int d, float scale, int causal, int diag_offset, int dtype, fa_stream_t stream) {
+  int rc = check_shape(B, Hq, Hkv, N, d, scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return FA_OK;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID;
+  // offsets beyond +-N change nothing; clamping keeps the kernel's index sums in range
+  const int shift = causal ? std::max(-N, std::min(N, diag_offset)) : 0;
+  int dev = 0;
+  if ((rc = check_device(&dev)) != FA_OK) return rc;
+  if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_fwd_bf16_2tile<64>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, shift);
+    case 128: return launch_fwd_bf16_2tile<128>(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, shift);
+    default: return launch_fwd_bf16_d256(q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, s, shift);
+  }
+}
+
+int fa_merge_partials(const void* o_parts, const float* lse_parts, int n_parts, long long rows, void* o, float* lse,
+                      int d, int dtype, fa_stream_t stream) {
+  if (n_parts < 1 || rows < 0 || (d != 64 && d != 128 && d != 256)) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_INVALID;
+  if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (rows == 0) return FA_OK;
+  if (rows > (1LL << 40) / n_parts) return FA_ERR_INVALID;
+  for (const void* ptr : {o_parts, static_cast<const void*>(lse_parts), static_cast<const void*>(o),
+                          static_cast<const void*>(lse)})
+    if (!aligned16(ptr)) return FA_ERR_INVALID;
+  // the output may not overlap the inputs (every thread reads all parts of
+  // its columns before writing, but the LSE of a row is read by all of its
+  // threads and written by one)
+  const auto lo = [](const void* ptr) { return reinterpret_cast<uintptr_t>(ptr); };
+  const uintptr_t in0 = lo(o_parts), in1 = in0 + static_cast<uintptr_t>(n_parts) * rows * d * 2;
+  const uintptr_t l0 = lo(lse_parts), l1 = l0 + static_cast<uintptr_t>(n_parts) * rows * 4;
+  const uintptr_t out0 = lo(o), out1 = out0 + static_cast<uintptr_t>(rows) * d * 2;
+  const uintptr_t lo0 = lo(lse), lo1 = lo0 + static_cast<uintptr_t>(rows) * 4;
+  for (const auto& a : {std::make_pair(out0, out1), std::make_pair(lo0, lo1)})
+    for (const auto& b : {std::make_pair(in0, in1), std::make_pair(l0, l1)})
+      if (a.first < b.second && b.first < a.second) return FA_ERR_INVALID;
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != FA_OK) return rc;
+  if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
+  int num_sms = 0;
+  if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_merge<64>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
+    case 128: return launch_merge<128>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
+    default: return launch_merge<256>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
+  }
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {

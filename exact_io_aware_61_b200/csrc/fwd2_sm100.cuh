@@ -62,6 +62,10 @@ struct Fwd2Params {
   const int* cu_q;
   const int* cu_k;
   int batch, total_q, total_k, max_seqlen_q;
+  // Causal diagonal moved by diag_shift keys: query i (at key position
+  // k_len - q_len + i) sees key j iff j <= k_len - q_len + i + diag_shift.
+  // Negative shifts leave rows with no visible key: O = 0, LSE = -inf.
+  int diag_shift;
 };
 
 constexpr int kStatusInvalid = 1;  // equals FA_ERR_INVALID: sequence offsets inconsistent with the sizes given
@@ -177,18 +181,33 @@ __global__ void __launch_bounds__(384, 1)
     bh_kv = b * p.Hkv + hq / (p.Hq / p.Hkv);
     q_len = k_len = p.N;
   }
-  // query i of the (sequence's) tile sits at key position kv_off + i: the
-  // last positions when a sequence has fewer queries than keys
-  const int kv_off = k_len - q_len;
+  // query i of the (sequence's) tile sees keys up to kv_off + i: the last
+  // positions when a sequence has fewer queries than keys, moved by the shift
+  const int kv_off = k_len - q_len + p.diag_shift;
   const int q0 = pair * 2 * C::BM;
   const int n_kv_total = (k_len + C::BN - 1) / C::BN;
   int n_t[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int qs = q0 + t * C::BM;
-    n_t[t] = qs < q_len ? (p.causal ? min((kv_off + qs + C::BM - 1) / C::BN + 1, n_kv_total) : n_kv_total) : 0;
+    const int last_key = kv_off + qs + C::BM - 1;  // causal: the last key any row of the tile sees
+    n_t[t] = qs >= q_len ? 0 : !p.causal ? n_kv_total : last_key < 0 ? 0 : min(last_key / C::BN + 1, n_kv_total);
   }
   const int n_max = max(n_t[0], n_t[1]);
+  if (n_max == 0) {
+    // causal with a negative shift: no row of either tile sees a key
+    if (warp < 8) {
+      const int row = q0 + (warp >> 2) * C::BM + (threadIdx.x & 127);
+      if (row < q_len) {
+        const size_t o_index = VARLEN ? static_cast<size_t>(q_tok + row) * p.Hq + hq : static_cast<size_t>(bh) * p.N + row;
+        uint4* dst = reinterpret_cast<uint4*>(p.o + o_index * HD);
+#pragma unroll
+        for (int i = 0; i < HD / 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+        p.lse[o_index] = -INFINITY;
+      }
+    }
+    return;
+  }
   // TMA coordinates (y, z) of query row 0 and of key row 0
   const int qy = VARLEN ? hq : 0, qz = VARLEN ? q_tok : bh;
   const int ky = VARLEN ? bh_kv : 0, kz = VARLEN ? k_tok : bh_kv;
@@ -372,12 +391,14 @@ __global__ void __launch_bounds__(384, 1)
         m_ref = mx;
       } else if (__any_sync(0xffffffffu, mx > m_ref + C::RESCALE_THRESHOLD)) {
         const float m_new = fmaxf(m_ref, mx);
-        alpha = ex2_approx(m_ref - m_new);
+        alpha = m_new == -INFINITY ? 1.f : ex2_approx(m_ref - m_new);
         m_ref = m_new;
         rescale = true;
       }
-      // p = 2^(s * scale * log2 e - m), packed to bf16 over the S columns
-      const uint64_t negm2 = pack2(-m_ref, -m_ref);
+      // p = 2^(s * scale * log2 e - m), packed to bf16 over the S columns; a
+      // row that sees no key (m = -inf) takes m = 0, so its p are all 0
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+      const uint64_t negm2 = pack2(-m_use, -m_use);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[64];
 #pragma unroll
@@ -426,7 +447,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (n > 0 && ok && warp_wait(smem_u32(&bar_odone[t]), (n - 1) & 1, wc)) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;  // l = 0: the row saw no key
       const bool live = row < q_len;
       const size_t o_index = VARLEN ? static_cast<size_t>(q_tok + (live ? row : 0)) * p.Hq + hq
                                     : static_cast<size_t>(bh) * p.N + (live ? row : 0);
@@ -446,7 +467,14 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 4; ++i) dst[i] = w[i];
         }
       }
-      if (live) p.lse[o_index] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+      if (live) p.lse[o_index] = l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    } else if (n == 0 && ok && row < q_len) {
+      // causal with a negative shift: no row of this tile sees a key
+      const size_t o_index = VARLEN ? static_cast<size_t>(q_tok + row) * p.Hq + hq : static_cast<size_t>(bh) * p.N + row;
+      uint4* dst = reinterpret_cast<uint4*>(p.o + o_index * HD);
+#pragma unroll
+      for (int i = 0; i < HD / 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+      p.lse[o_index] = -INFINITY;
     }
   }
 

@@ -54,6 +54,9 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e)
   int causal;
   unsigned long long timeout_ns;
+  // causal: query i sees key j iff j <= i + diag_shift; a row that sees no
+  // key gets O = 0, LSE = -inf
+  int diag_shift;
 };
 
 template <int HD>
@@ -87,7 +90,19 @@ __global__ void __launch_bounds__(192, 1)
   const int bh_kv = b * p.Hkv + hq / (p.Hq / p.Hkv);
   const int q0 = qt * C::BM;
   const int n_kv_total = (p.N + C::BN - 1) / C::BN;
-  const int n_kv = p.causal ? min(qt + 1, n_kv_total) : n_kv_total;
+  const int last_key = q0 + C::BM - 1 + p.diag_shift;  // causal: the last key any row of the tile sees
+  const int n_kv = !p.causal ? n_kv_total : last_key < 0 ? 0 : min(last_key / C::BN + 1, n_kv_total);
+  if (n_kv == 0) {
+    // causal with a negative shift: no row of the tile sees a key
+    const int row = q0 + threadIdx.x;
+    if (threadIdx.x < C::BM && row < p.N) {
+      uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * p.N + row) * HD);
+#pragma unroll
+      for (int i = 0; i < HD / 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+      p.lse[static_cast<size_t>(bh) * p.N + row] = -INFINITY;
+    }
+    return;
+  }
 
   WaitCtl wc{&abort_flag, p.timeout_ns};
 
@@ -214,9 +229,9 @@ __global__ void __launch_bounds__(192, 1)
         for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
       }
       const int key0 = j * C::BN;
-      const bool diag = p.causal && (key0 + C::BN > q0);
+      const bool diag = p.causal && (key0 + C::BN > q0 + p.diag_shift);
       if (diag || key0 + C::BN > p.N) {
-        const int lim = min(p.causal ? row + 1 : p.N, p.N) - key0;  // keys [key0, key0+lim) visible
+        const int lim = min(p.causal ? row + p.diag_shift + 1 : p.N, p.N) - key0;  // keys [key0, key0+lim) visible
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= lim) s[c] = -INFINITY;
@@ -231,7 +246,7 @@ __global__ void __launch_bounds__(192, 1)
         const bool need = mx > m_ref + C::RESCALE_THRESHOLD;
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = fmaxf(m_ref, mx);
-          const float alpha = ex2_approx(m_ref - m_new);
+          const float alpha = m_new == -INFINITY ? 1.f : ex2_approx(m_ref - m_new);
           // o was last written by P_{j-1} V_{j-1}; wait for it, then rescale.
           if (!warp_wait(smem_u32(&bar_odone), (j - 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
@@ -248,7 +263,7 @@ __global__ void __launch_bounds__(192, 1)
           m_ref = m_new;
         }
       }
-      const float neg_m = -m_ref;
+      const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;  // a row that sees no key: every p = 0
       float sum = 0.f;
       uint32_t pk[64];
 #pragma unroll
@@ -272,7 +287,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (ok && warp_wait(smem_u32(&bar_odone), (n_kv - 1) & 1, wc)) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;  // l = 0: the row saw no key
       const bool live = row < p.N;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (live ? row : 0)) * HD;
 #pragma unroll
@@ -290,7 +305,9 @@ __global__ void __launch_bounds__(192, 1)
           for (int i = 0; i < 4; ++i) dst[i] = w[i];
         }
       }
-      if (live) p.lse[static_cast<size_t>(bh) * p.N + row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+      if (live)
+        p.lse[static_cast<size_t>(bh) * p.N + row] =
+            l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
   }
 

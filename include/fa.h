@@ -100,6 +100,50 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
            int dtype, fa_stream_t stream);
 
 /*
+ * fa_fwd_partial -- fa_fwd over one block of a longer sequence, for attention
+ * sharded over the sequence dimension.
+ *
+ *   arguments as fa_fwd; dtype FA_BF16 only (FA_F32 returns
+ *   FA_ERR_UNSUPPORTED)
+ *   diag_offset: with causal = 1, query row i sees key row j iff
+ *                j <= i + diag_offset (0 gives fa_fwd; values beyond +-N
+ *                act as +-N); ignored when causal = 0
+ * A row that sees no key (causal, i + diag_offset < 0) gets O = 0 and
+ * LSE = -inf. The outputs are the block's own softmax, normalised over its
+ * keys, with the LSE that fa_merge_partials needs to combine blocks: the
+ * pages name parallelism over the sequence dimension (synthetic.wiki
+ * "FlashAttention: attention's bottleneck is the wire, not the maths",
+ * "Versions, and what the numbers say") and the rescale rule that makes
+ * the merge exact ("A pinch of math"). With the striped assignment (token t
+ * on device t mod W), device r's queries against device c's keys are this
+ * call with diag_offset 0 for c <= r and -1 for c > r. Returns fa_status.
+ */
+FA_API int fa_fwd_partial(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                   int diag_offset, int dtype, fa_stream_t stream);
+
+/*
+ * fa_merge_partials -- combine normalised outputs of disjoint key sets.
+ *
+ *   o_parts [n_parts][rows][d]   input (bf16): part p's output for each row
+ *   lse_parts [n_parts][rows]    input, float32: part p's LSE (-inf: the
+ *                                part saw no key of that row)
+ *   o [rows][d]                  output (bf16)
+ *   lse [rows]                   output, float32, natural log
+ *   n_parts >= 1, rows >= 0, d in {64, 128, 256}, dtype FA_BF16
+ * With M = max_p LSE_p: L = sum_p exp(LSE_p - M), O = sum_p exp(LSE_p - M)
+ * O_p / L, LSE = M + ln L, in float32 ("A pinch of math": the rescale of
+ * the running state, applied to states already divided by l). Rows whose
+ * parts are all -inf get O = 0, LSE = -inf. rows counts (batch, head,
+ * query) triples, so an fa_fwd_partial output [B][Hq][N][d] is
+ * rows = B * Hq * N. The outputs may not overlap the inputs
+ * (FA_ERR_INVALID). Returns fa_status.
+ */
+FA_API int fa_merge_partials(const void* o_parts, const float* lse_parts, int n_parts,
+                      long long rows, void* o, float* lse, int d, int dtype,
+                      fa_stream_t stream);
+
+/*
  * fa_fwd_varlen -- forward pass over a packed batch of sequences of
  * different lengths, or over strided "BNHD" tensors.
  *
