@@ -300,23 +300,30 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
   return launch_status(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<HD, true>));
 }
 
-template <int HD>
-int launch_merge(const void* o_parts, const float* lse_parts, int n_parts, long long rows, void* o, float* lse,
-                 int num_sms, cudaStream_t stream) {
+template <int HD, int UNROLL>
+int launch_merge_u(const void* o_parts, const float* lse_parts, int n_parts, long long rows, void* o, float* lse,
+                   int num_sms, cudaStream_t stream) {
   constexpr int TPR = HD / 8;
   const long long threads = rows * TPR;
   const long long want = (threads + fa::MergeCfg::THREADS - 1) / fa::MergeCfg::THREADS;
   // grid-stride over rows with exactly the blocks that are resident at once
   // (a second, partial wave would leave its blocks a full share of rows)
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fa::fa_merge_partials_kernel<HD>,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fa::fa_merge_partials_kernel<HD, UNROLL>,
                                                     fa::MergeCfg::THREADS, 0) != cudaSuccess ||
       per_sm < 1)
     return FA_ERR_CUDA;
   const long long blocks = std::min<long long>(want, static_cast<long long>(per_sm) * num_sms);
-  fa::fa_merge_partials_kernel<HD><<<static_cast<unsigned>(blocks), fa::MergeCfg::THREADS, 0, stream>>>(
+  fa::fa_merge_partials_kernel<HD, UNROLL><<<static_cast<unsigned>(blocks), fa::MergeCfg::THREADS, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o_parts), lse_parts, n_parts, rows, static_cast<__nv_bfloat16*>(o), lse);
   return launch_status();
+}
+
+template <int HD>
+int launch_merge(const void* o_parts, const float* lse_parts, int n_parts, long long rows, void* o, float* lse,
+                 int num_sms, cudaStream_t stream) {
+  return n_parts <= 4 ? launch_merge_u<HD, 4>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, stream)
+                      : launch_merge_u<HD, 8>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, stream);
 }
 
 template <int HD>

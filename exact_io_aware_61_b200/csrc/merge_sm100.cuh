@@ -27,7 +27,6 @@ namespace fa {
 
 struct MergeCfg {
   static constexpr int THREADS = 256;
-  static constexpr int UNROLL = 8;      // parts whose loads are in flight together
   static constexpr int MIN_BLOCKS = 8;  // 2048 resident threads per SM (32 registers each)
 };
 
@@ -47,7 +46,9 @@ FA_DEV float ld_nc_f32(const float* ptr) {
   return r;
 }
 
-template <int HD>
+// UNROLL: parts whose loads are in flight together (4 or 8, the host picks
+// the smaller when it covers every part)
+template <int HD, int UNROLL>
 __global__ void __launch_bounds__(MergeCfg::THREADS, MergeCfg::MIN_BLOCKS)
     fa_merge_partials_kernel(const __nv_bfloat16* __restrict__ o_parts, const float* __restrict__ lse_parts,
                              int n_parts, long long rows, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
@@ -61,15 +62,15 @@ __global__ void __launch_bounds__(MergeCfg::THREADS, MergeCfg::MIN_BLOCKS)
     // pass 1: the row's largest LSE (all loads independent, the row's threads
     // read the same addresses)
     float M = -INFINITY;
-    for (int q0 = 0; q0 < n_parts; q0 += MergeCfg::UNROLL) {
-      float lq[MergeCfg::UNROLL];
+    for (int q0 = 0; q0 < n_parts; q0 += UNROLL) {
+      float lq[UNROLL];
 #pragma unroll
-      for (int u = 0; u < MergeCfg::UNROLL; ++u)
+      for (int u = 0; u < UNROLL; ++u)
         lq[u] = ld_nc_f32(lse_parts + static_cast<long long>(min(q0 + u, n_parts - 1)) * rows + row);
 #pragma unroll
-      for (int u = 0; u < MergeCfg::UNROLL; ++u) asm volatile("" : "+f"(lq[u]));
+      for (int u = 0; u < UNROLL; ++u) asm volatile("" : "+f"(lq[u]));
 #pragma unroll
-      for (int u = 0; u < MergeCfg::UNROLL; ++u) M = fmaxf(M, lq[u]);  // a repeated last part changes no max
+      for (int u = 0; u < UNROLL; ++u) M = fmaxf(M, lq[u]);  // a repeated last part changes no max
     }
     float acc[8];
 #pragma unroll
@@ -80,11 +81,11 @@ __global__ void __launch_bounds__(MergeCfg::THREADS, MergeCfg::MIN_BLOCKS)
       // pass 2: UNROLL parts at a time, every load issued before any is used;
       // past the last part the index is clamped (a valid address) and the
       // weight is 0, and a part with LSE = -inf weighs 0 whatever its O holds
-      for (int q0 = 0; q0 < n_parts; q0 += MergeCfg::UNROLL) {
-        float lq[MergeCfg::UNROLL];
-        uint4 x[MergeCfg::UNROLL];
+      for (int q0 = 0; q0 < n_parts; q0 += UNROLL) {
+        float lq[UNROLL];
+        uint4 x[UNROLL];
 #pragma unroll
-        for (int u = 0; u < MergeCfg::UNROLL; ++u) {
+        for (int u = 0; u < UNROLL; ++u) {
           const long long idx = static_cast<long long>(min(q0 + u, n_parts - 1)) * rows + row;
           lq[u] = ld_nc_f32(lse_parts + idx);
           x[u] = ld_nc_v4(o_parts + idx * HD + c8);
@@ -92,10 +93,10 @@ __global__ void __launch_bounds__(MergeCfg::THREADS, MergeCfg::MIN_BLOCKS)
         // every use below depends on these (empty, ordered) statements, which
         // come after the last load: the batch is issued before it is waited on
 #pragma unroll
-        for (int u = 0; u < MergeCfg::UNROLL; ++u)
+        for (int u = 0; u < UNROLL; ++u)
           asm volatile("" : "+r"(x[u].x), "+r"(x[u].y), "+r"(x[u].z), "+r"(x[u].w), "+f"(lq[u]));
 #pragma unroll
-        for (int u = 0; u < MergeCfg::UNROLL; ++u) {
+        for (int u = 0; u < UNROLL; ++u) {
           const bool use = q0 + u < n_parts && lq[u] != -INFINITY;
           const float w = use ? ex2_approx(fmaf(lq[u], kLog2e, -m2)) : 0.f;
           L += w;

@@ -90,6 +90,7 @@ __all__ = [
     "score_matrix_bytes",
     "attention_forward_kvcache",
     "attention_forward_varlen",
+    "attention_backward_varlen",
     "partial_state",
     "merge_partial_states",
     "attention_forward_positions",
@@ -454,3 +455,43 @@ def merge_outputs(os, lses):
     os, lses = _f64(os), _f64(lses)
     finite = np.isfinite(lses)
     return merge_partial_states(lses, finite.astype(np.float64), np.where(finite[..., None], os, 0.0))
+
+
+def attention_backward_varlen(q, k, v, do, cu_q, cu_k, scale: float, causal: bool):
+    """Gradients of :func:`attention_forward_varlen` for the upstream gradient ``do``.
+
+    Layouts as in the forward: ``q``, ``do`` are ``[total_q, Hq, d]``, ``k``,
+    ``v`` are ``[total_k, Hkv, d]``. Each sequence is its own problem, with its
+    queries at its last positions; the formulas are those of
+    :func:`attention_backward`, per sequence and head, and dK, dV sum over the
+    query heads of a KV head's group. A key no query sees gets zero gradient.
+    Returns ``(dQ [total_q, Hq, d], dK [total_k, Hkv, d], dV [total_k, Hkv, d])``.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    do = _f64(do)
+    cu_q = np.asarray(cu_q, dtype=np.int64)
+    cu_k = np.asarray(cu_k, dtype=np.int64)
+    if cu_q.shape != cu_k.shape or cu_q[0] != 0 or cu_k[0] != 0:
+        raise ValueError("cu_q and cu_k must start at 0 and have one entry per sequence boundary")
+    Hq, Hkv = q.shape[1], k.shape[1]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for sq in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[sq], cu_q[sq + 1], cu_k[sq], cu_k[sq + 1]
+        if q1 - q0 > k1 - k0:
+            raise ValueError("a sequence has more queries than keys")
+        pos = (k1 - k0) - (q1 - q0) + np.arange(q1 - q0)
+        for h in range(Hq):
+            hk = kv_head_of(h, Hq, Hkv)
+            qs, ks, vs, dos = q[q0:q1, h], k[k0:k1, hk], v[k0:k1, hk], do[q0:q1, h]
+            p = softmax_rows(masked_scores(qs, ks, scale, causal, rows=pos))[0]
+            dv[k0:k1, hk] += p.T @ dos
+            dp = dos @ vs.T
+            D = np.sum(dos * (p @ vs), axis=1)
+            ds = score_gradient(p, dp, D)
+            dq[q0:q1, h] = scale * (ds @ ks)
+            dk[k0:k1, hk] += scale * (ds.T @ qs)
+    return dq, dk, dv

@@ -417,7 +417,53 @@ def check_striped_shards_merge_to_full(o):
             assert np.max(np.abs(ml - fl[:, :, r::W].reshape(-1))) < 1e-13
 
 
+
+def check_varlen_backward_square_sequences_are_the_square_backward(o):
+    # Sequences with as many queries as keys are each the (pinned) square
+    # backward of that sequence alone.
+    rng = np.random.default_rng(107)
+    lens = [6, 1, 9]
+    cu = np.cumsum([0] + lens)
+    q, k, v, do = (rng.standard_normal((cu[-1], h, 4)) for h in (4, 2, 2, 4))
+    for causal in (False, True):
+        dq, dk, dv = o.attention_backward_varlen(q, k, v, do, cu, cu, 0.6, causal)
+        for s in range(3):
+            sl = slice(cu[s], cu[s + 1])
+            per = [x[sl].transpose(1, 0, 2)[None] for x in (q, k, v, do)]
+            rq, rk, rv, _ = o.attention_backward(*per, 0.6, causal)
+            assert np.max(np.abs(dq[sl] - rq[0].transpose(1, 0, 2))) < 1e-13
+            assert np.max(np.abs(dk[sl] - rk[0].transpose(1, 0, 2))) < 1e-13
+            assert np.max(np.abs(dv[sl] - rv[0].transpose(1, 0, 2))) < 1e-13
+
+
+def check_varlen_backward_finite_differences(o):
+    # Central differences of L = sum(O * G) through the (pinned) varlen
+    # forward, on a pack whose sequences have fewer queries than keys (the
+    # queries sit at the last positions) and GQA.
+    rng = np.random.default_rng(109)
+    cq, ck = np.array([0, 2, 5]), np.array([0, 4, 7])
+    q, k, v = rng.standard_normal((5, 2, 3)), rng.standard_normal((7, 1, 3)), rng.standard_normal((7, 1, 3))
+    g = rng.standard_normal((5, 2, 3))
+    for causal in (False, True):
+        dq, dk, dv = o.attention_backward_varlen(q, k, v, g, cq, ck, 0.8, causal)
+        for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            num = np.zeros_like(x)
+            for idx in np.ndindex(*x.shape):
+                xp, xm = x.copy(), x.copy()
+                xp[idx] += 1e-6
+                xm[idx] -= 1e-6
+                args = {"q": q, "k": k, "v": v}
+                args[name] = xp
+                fp = np.sum(o.attention_forward_varlen(args["q"], args["k"], args["v"], cq, ck, 0.8, causal)[0] * g)
+                args[name] = xm
+                fm = np.sum(o.attention_forward_varlen(args["q"], args["k"], args["v"], cq, ck, 0.8, causal)[0] * g)
+                num[idx] = (fp - fm) / 2e-6
+            assert np.max(np.abs(num - grad)) < 1e-7, name
+
+
 ALL_CHECKS = [
+    check_varlen_backward_square_sequences_are_the_square_backward,
+    check_varlen_backward_finite_differences,
     check_positions_reduce_to_square_and_kvcache,
     check_positions_brute_force,
     check_striped_shards_merge_to_full,
@@ -481,6 +527,21 @@ def _mut_transposed_keys(q_bh, k_bh, scale, causal, rows=None, keys=None):  # K^
         kpos = np.arange(s.shape[1]) if keys is None else np.asarray(keys)
         s = np.where(kpos[None, :] <= qpos[:, None], s, -np.inf)
     return s
+
+
+def _mut_varlen_backward_top_left(q, k, v, do, cu_q, cu_k, scale, causal):  # queries placed at positions 0..
+    q, k, v, do = (np.asarray(x, float) for x in (q, k, v, do))
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for s in range(len(cu_q) - 1):
+        sq, sk = slice(cu_q[s], cu_q[s + 1]), slice(cu_k[s], cu_k[s + 1])
+        for h in range(q.shape[1]):
+            hk = ORACLE.kv_head_of(h, q.shape[1], k.shape[1])
+            p = ORACLE.softmax_rows(ORACLE.masked_scores(q[sq, h], k[sk, hk], scale, causal))[0]
+            dv[sk, hk] += p.T @ do[sq, h]
+            ds = ORACLE.score_gradient(p, do[sq, h] @ v[sk, hk].T, np.sum(do[sq, h] * (p @ v[sk, hk]), axis=1))
+            dq[sq, h] = scale * (ds @ k[sk, hk])
+            dk[sk, hk] += scale * (ds.T @ q[sq, h])
+    return dq, dk, dv
 
 
 def _mut_positions_ignore_keys(q, k, v, q_pos, k_pos, scale, causal):  # key positions taken as 0..Nk-1
@@ -553,6 +614,7 @@ MUTATIONS = [
     ("attention_forward_varlen", _mut_varlen_leak),
     ("attention_forward_positions", _mut_positions_ignore_keys),
     ("merge_outputs", _mut_merge_outputs_plain_mean),
+    ("attention_backward_varlen", _mut_varlen_backward_top_left),
 ]
 
 
