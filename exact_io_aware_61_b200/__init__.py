@@ -18,11 +18,15 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     FAError,
     backward,
+    backward_bnhd,
+    backward_varlen,
     fa_bwd,
     fa_bwd_main,
     fa_bwd_dq,
     fa_bwd_noalloc,
     fa_bwd_prep,
+    fa_bwd_varlen,
+    fa_bwd_varlen_workspace_size,
     fa_bwd_workspace_size,
     fa_fwd,
     fa_fwd_kvcache,

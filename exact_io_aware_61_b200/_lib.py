@@ -31,6 +31,8 @@ EXPORTED = (
     "fa_bwd_dq",
     "fa_bwd_noalloc",
     "fa_bwd_workspace_size",
+    "fa_bwd_varlen",
+    "fa_bwd_varlen_workspace_size",
     "fa_fwd_kvcache",
     "fa_fwd_kvcache_workspace_size",
     "fa_status_string",
@@ -79,6 +81,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_bwd_dq.restype = i
         lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
         lib.fa_bwd_noalloc.restype = i
+        lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i,
+                                      vp, sz, i, vp]
+        lib.fa_bwd_varlen.restype = i
+        lib.fa_bwd_varlen_workspace_size.argtypes = [i, i, i, i, i, i]
+        lib.fa_bwd_varlen_workspace_size.restype = sz
         lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i]
         lib.fa_bwd_workspace_size.restype = sz
         lib.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, f, i, i, vp]
@@ -205,6 +212,57 @@ def forward_bnhd(q, k, v, causal: bool = False, scale: float | None = None, stre
     o, lse = forward_varlen(q.reshape(B * N, Hq, d), k.reshape(B * N, k.shape[2], d), v.reshape(B * N, v.shape[2], d),
                             offs, offs, N, causal, scale, stream)
     return o.view(B, N, Hq, d), lse.view(B, N, Hq)
+
+
+def fa_bwd_varlen_workspace_size(batch: int, total_q: int, total_k: int, Hq: int, Hkv: int, d: int) -> int:
+    return int(load().fa_bwd_varlen_workspace_size(batch, total_q, total_k, Hq, Hkv, d))
+
+
+def fa_bwd_varlen(q, k, v, o, lse, do, dq, dk, dv, cu_q, cu_k, max_seqlen_q: int, max_seqlen_k: int, workspace,
+                  causal: bool, scale: float, stream=None) -> None:
+    """Call ``fa_bwd_varlen``: packed layouts as ``fa_fwd_varlen`` (q, o, do, dq [total_q, Hq, d]; k, v, dk, dv
+    [total_k, Hkv, d]; lse [total_q, Hq] f32), int32 offsets cu_q, cu_k, a uint8 workspace."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse), ("do", do), ("dq", dq), ("dk", dk),
+                    ("dv", dv), ("cu_q", cu_q), ("cu_k", cu_k)):
+        _check_tensor(name, t, q.device)
+    if cu_q.dtype != torch.int32 or cu_k.dtype != torch.int32:
+        raise TypeError("cu_q and cu_k must be int32")
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    ws_ptr, ws_bytes = _ws(workspace)
+    rc = load().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                              _ptr(cu_q), _ptr(cu_k), cu_q.numel() - 1, int(max_seqlen_q), int(max_seqlen_k), total_q,
+                              total_k, Hq, Hkv, d, float(scale), int(bool(causal)), ws_ptr, ws_bytes,
+                              _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_varlen")
+
+
+def backward_varlen(q, k, v, o, lse, do, cu_q, cu_k, max_seqlen_q: int, max_seqlen_k: int, causal: bool = False,
+                    scale: float | None = None, stream=None):
+    """Allocate dQ, dK, dV and the workspace with torch and run ``fa_bwd_varlen``."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nbytes = fa_bwd_varlen_workspace_size(cu_q.numel() - 1, q.shape[0], k.shape[0], q.shape[1], k.shape[1],
+                                          q.shape[2])
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    fa_bwd_varlen(q, k, v, o, lse, do, dq, dk, dv, cu_q, cu_k, max_seqlen_q, max_seqlen_k, ws, causal, scale, stream)
+    return dq, dk, dv
+
+
+def backward_bnhd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, stream=None):
+    """Backward over strided [B, N, H, d] tensors (``o``, ``lse`` as ``forward_bnhd`` returns them).
+
+    Returns ``(dq, dk, dv)`` in the same [B, N, H, d] layouts; runs ``fa_bwd_varlen`` with offsets 0, N, ..., B*N.
+    """
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    offs = torch.arange(0, (B + 1) * N, N, dtype=torch.int32, device=q.device)
+    dq, dk, dv = backward_varlen(q.reshape(B * N, Hq, d), k.reshape(B * N, Hkv, d), v.reshape(B * N, Hkv, d),
+                                 o.reshape(B * N, Hq, d), lse.reshape(B * N, Hq), do.reshape(B * N, Hq, d), offs, offs,
+                                 N, N, causal, scale, stream)
+    return dq.view(B, N, Hq, d), dk.view(B, N, Hkv, d), dv.view(B, N, Hkv, d)
 
 
 def fa_bwd_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:

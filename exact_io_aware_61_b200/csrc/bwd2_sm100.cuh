@@ -42,6 +42,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include "sm100_ptx.cuh"
+#include "bwd_sm100.cuh"  // ws_seq_base
 
 namespace fa {
 
@@ -90,10 +91,24 @@ struct Bwd2Params {
   float scale;
   int causal;
   unsigned long long timeout_ns;
+  // Packed variable-length batches (the VARLEN kernel only): sequence s owns
+  // query tokens cu_q[s] .. cu_q[s+1]-1 of Q, dO [total_q][Hq][d] and key
+  // tokens cu_k[s] .. cu_k[s+1]-1 of K, V, dK, dV [total_k][Hkv][d]; its
+  // queries are its last positions. The dQ accumulator is laid out like Q.
+  // Each query head's workspace row (Npad floats) holds sequence s from
+  // ws_seq_base(s), so every 128-row tile starts on a 16-byte boundary.
+  // num_tiles covers the longest key sequence.
+  const int* cu_q;
+  const int* cu_k;
+  int batch, total_q, total_k, max_seqlen_q, max_seqlen_k;
 };
 
+
 // 16 warps, 4 per SM sub-partition: 16384 / 128 -> 128 registers at launch.
-template <int HD>
+// VARLEN: packed variable-length batches (see Bwd2Params); the tensor maps are
+// then rank-3 views {d, heads, tokens} with a {64 or 32, 1, 128} box, which
+// lands in shared memory like the dense box.
+template <int HD, bool VARLEN = false>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd2_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -120,27 +135,74 @@ __global__ void __launch_bounds__(512, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Block order: groups of KV_GROUP (batch, KV head) pairs, whose K, V, Q and
-  // dO stay in L2 together; inside a group the key tiles go heaviest first
-  // (tile 0 has the most work when causal), each over the group's heads and
-  // head slices, so the last blocks to start are the shortest.
-  const int per_kv = p.num_tiles * p.head_split;
-  const int grp = static_cast<int>(blockIdx.x) / (C::KV_GROUP * per_kv);
-  const int in_grp = min(C::KV_GROUP, p.BHkv - grp * C::KV_GROUP);
-  const int r0 = static_cast<int>(blockIdx.x) - grp * C::KV_GROUP * per_kv;
-  const int kt = r0 / (in_grp * p.head_split);
-  const int r1 = r0 - kt * in_grp * p.head_split;
-  const int bhkv = grp * C::KV_GROUP + r1 / p.head_split;
-  const int slice = r1 - (r1 / p.head_split) * p.head_split;
+  // Block order (dense): groups of KV_GROUP (batch, KV head) pairs, whose K,
+  // V, Q and dO stay in L2 together; inside a group the key tiles go
+  // heaviest first (tile 0 has the most work when causal), each over the
+  // group's heads and head slices, so the last blocks to start are the
+  // shortest. Variable-length: every (sequence, KV head, slice) at one key
+  // tile index, tile indices from 0 up; CTAs past their sequence's keys
+  // leave at once.
+  int kt, bhkv, slice, b, hkv;
+  int q_len, k_len, q_tok = 0, k_tok = 0, ws_base = 0;
+  if constexpr (VARLEN) {
+    const int per_kt = p.batch * p.Hkv * p.head_split;
+    kt = static_cast<int>(blockIdx.x) / per_kt;
+    const int r0 = static_cast<int>(blockIdx.x) - kt * per_kt;
+    b = r0 / (p.Hkv * p.head_split);
+    const int r1 = r0 - b * p.Hkv * p.head_split;
+    hkv = r1 / p.head_split;
+    slice = r1 - hkv * p.head_split;
+    bhkv = hkv;
+    q_tok = p.cu_q[b];
+    k_tok = p.cu_k[b];
+    q_len = p.cu_q[b + 1] - q_tok;
+    k_len = p.cu_k[b + 1] - k_tok;
+    const bool bad = q_tok < 0 || k_tok < 0 || q_len < 0 || k_len < q_len || q_len > p.max_seqlen_q ||
+                     k_len > p.max_seqlen_k || q_tok + q_len > p.total_q || k_tok + k_len > p.total_k;
+    if (bad) {
+      if (threadIdx.x == 0) atomicCAS(&g_status, 0, kStatusInvalid);
+      return;
+    }
+    if (kt * 128 >= k_len) return;  // no keys of this sequence here
+    ws_base = ws_seq_base(q_tok, b);
+  } else {
+    const int per_kv = p.num_tiles * p.head_split;
+    const int grp = static_cast<int>(blockIdx.x) / (C::KV_GROUP * per_kv);
+    const int in_grp = min(C::KV_GROUP, p.BHkv - grp * C::KV_GROUP);
+    const int r0 = static_cast<int>(blockIdx.x) - grp * C::KV_GROUP * per_kv;
+    kt = r0 / (in_grp * p.head_split);
+    const int r1 = r0 - kt * in_grp * p.head_split;
+    bhkv = grp * C::KV_GROUP + r1 / p.head_split;
+    slice = r1 - (r1 / p.head_split) * p.head_split;
+    b = bhkv / p.Hkv;
+    hkv = bhkv - b * p.Hkv;
+    q_len = k_len = p.N;
+  }
   const int k0 = kt * 128;
-  const int b = bhkv / p.Hkv;
-  const int hkv = bhkv - b * p.Hkv;
   const int group = p.Hq / p.Hkv;
   const int heads = group / p.head_split;  // query heads of this CTA's slice
   const int h_first = slice * heads;
-  const int i_begin = p.causal ? kt : 0;
-  const int per_head = p.num_tiles - i_begin;
-  const int steps = heads * per_head;
+  // query i of the sequence sits at key position kv_off + i (its last
+  // positions when it has fewer queries than keys)
+  const int kv_off = k_len - q_len;
+  const int i_begin = p.causal ? max(0, (k0 - kv_off) / 128) : 0;  // first query tile that sees key tile kt
+  const int per_head = (q_len + 127) / 128 - i_begin;
+  const int steps = heads * max(per_head, 0);
+  if constexpr (VARLEN) {
+    if (steps == 0) {
+      // a sequence without queries: its keys get zero gradients (already
+      // zero in the f32 accumulators when the group is split)
+      if (p.head_split == 1 && threadIdx.x < 256) {
+        const int key = k0 + (threadIdx.x & 127);
+        if (key < k_len) {
+          __nv_bfloat16* out = (threadIdx.x < 128 ? p.dv : p.dk) + (static_cast<size_t>(k_tok + key) * p.Hkv + hkv) * HD;
+#pragma unroll
+          for (int i = 0; i < HD / 8; ++i) reinterpret_cast<uint4*>(out)[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      return;
+    }
+  }
 
   WaitCtl wc{&abort_flag, p.timeout_ns};
 
@@ -173,10 +235,17 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
+  // step t: query tile q0 of query head hq (dense: row bhq = b Hq + hq of the
+  // [B Hq] heads; variable-length: hq itself, the sequence being fixed)
   auto step_tile = [&](int t, int& bhq, int& q0) {
     const int hh = t / per_head;
     q0 = (i_begin + (t - hh * per_head)) * 128;
-    bhq = b * p.Hq + hkv * group + h_first + hh;
+    bhq = (VARLEN ? 0 : b * p.Hq) + hkv * group + h_first + hh;
+  };
+  // TMA coordinates (y, z) of row r of query head row bhq / of the key tile
+  auto q_yz = [&](int bhq, int r, int& y, int& z) {
+    y = VARLEN ? bhq : r;
+    z = VARLEN ? q_tok + r : bhq;
   };
 
   if (warp >= 12) {
@@ -187,9 +256,10 @@ __global__ void __launch_bounds__(512, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_do);
       mbar_arrive_expect_tx(smem_u32(&bar_kv), 2 * C::TILE);
+      const int ky = VARLEN ? hkv : k0, kz = VARLEN ? k_tok + k0 : bhkv;
       for (int c = 0; c < KCH; ++c) {
-        tma_load_3d(sK + c * 16384, &tm_k, smem_u32(&bar_kv), c * 64, k0, bhkv);
-        tma_load_3d(sV + c * 16384, &tm_v, smem_u32(&bar_kv), c * 64, k0, bhkv);
+        tma_load_3d(sK + c * 16384, &tm_k, smem_u32(&bar_kv), c * 64, ky, kz);
+        tma_load_3d(sV + c * 16384, &tm_v, smem_u32(&bar_kv), c * 64, ky, kz);
       }
       int q_issued = 0, do_issued = 0;
       for (int t = 0; t < steps; ++t) {
@@ -200,15 +270,17 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t qst = sQ + sq * C::QSTAGE_BYTES;
         const uint32_t qb = smem_u32(&bar_qfull[sq]);
         mbar_arrive_expect_tx(qb, C::QSTAGE_BYTES);
-        for (int c = 0; c < KCH; ++c) tma_load_3d(qst + c * 16384, &tm_q, qb, c * 64, q0, bhq);
-        const size_t roff = static_cast<size_t>(bhq) * p.Npad + q0;
+        int qy, qz;
+        q_yz(bhq, q0, qy, qz);
+        for (int c = 0; c < KCH; ++c) tma_load_3d(qst + c * 16384, &tm_q, qb, c * 64, qy, qz);
+        const size_t roff = static_cast<size_t>(bhq) * p.Npad + ws_base + q0;
         bulk_load(qst + C::TILE, p.ws_lse2 + roff, 512, qb);
         bulk_load(qst + C::TILE + 512, p.ws_delta + roff, 512, qb);
         q_issued = t + 1;
         if (!mbar_wait(smem_u32(&bar_doempty[sd]), ((t / DOST) & 1) ^ 1, wc)) break;
         const uint32_t db = smem_u32(&bar_dofull[sd]);
         mbar_arrive_expect_tx(db, C::TILE);
-        for (int c = 0; c < KCH; ++c) tma_load_3d(sDO + sd * C::TILE + c * 16384, &tm_do, db, c * 64, q0, bhq);
+        for (int c = 0; c < KCH; ++c) tma_load_3d(sDO + sd * C::TILE + c * 16384, &tm_do, db, c * 64, qy, qz);
         do_issued = t + 1;
       }
       // leave no copy in flight into shared memory (a bounded wait elsewhere
@@ -308,7 +380,7 @@ __global__ void __launch_bounds__(512, 1)
     const int cb = half * 64;           // first query column of this warpgroup
     const uint32_t lane_base = ((warp & 3) * 32u) << 16;
     const int key = k0 + tid;
-    const bool key_live = key < p.N;
+    const bool key_live = key < k_len;
     uint8_t* ds_row = gbase + (sDS - base) + half * 16384 + tid * 128;
     bool ok = true;
     for (int t = 0; t < steps; ++t) {
@@ -324,7 +396,11 @@ __global__ void __launch_bounds__(512, 1)
       // ---- P^T = exp2(S^T * scale * log2 e - LSE2), masked; kept in
       // registers too, since S^T(t+1) overwrites these columns once dV(t) has
       // read them
-      const bool diag = p.causal && (q0 == k0);
+      // some element of the tile is masked: a key after its query (causal),
+      // or, variable-length, a query past the sequence's end (its workspace
+      // row may belong to the next sequence, so the weight is zeroed here;
+      // dense padding rows have LSE = +inf and weigh 0 already)
+      const bool mask = VARLEN ? (p.causal && k0 + 127 > kv_off + q0) || q0 + 128 > q_len : p.causal && q0 == k0;
       uint32_t pk[32];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
@@ -339,10 +415,12 @@ __global__ void __launch_bounds__(512, 1)
           pv[1] = ex2_approx(fmaf(__uint_as_float(rr[4 * x + 1]), p.scale_log2, -L.y));
           pv[2] = ex2_approx(fmaf(__uint_as_float(rr[4 * x + 2]), p.scale_log2, -L.z));
           pv[3] = ex2_approx(fmaf(__uint_as_float(rr[4 * x + 3]), p.scale_log2, -L.w));
-          if (diag) {
+          if (mask) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (q0 + qa + e < key) pv[e] = 0.f;
+            for (int e = 0; e < 4; ++e) {
+              const int qi = q0 + qa + e;
+              if (VARLEN ? (p.causal && key > kv_off + qi) || qi >= q_len : qi < key) pv[e] = 0.f;
+            }
           }
           pk[u * 16 + 2 * x] = key_live ? pack_bf16x2(pv[0], pv[1]) : 0u;
           pk[u * 16 + 2 * x + 1] = key_live ? pack_bf16x2(pv[2], pv[3]) : 0u;
@@ -391,7 +469,8 @@ __global__ void __launch_bounds__(512, 1)
     // CTAs, f32 rows added into the accumulators
     if (ok && warp_wait(smem_u32(&bar_final), 0, wc)) {
       tc_fence_after();
-      const size_t row_off = (static_cast<size_t>(bhkv) * p.N + (key_live ? key : 0)) * HD;
+      const size_t row_off = VARLEN ? (static_cast<size_t>(k_tok + (key_live ? key : 0)) * p.Hkv + hkv) * HD
+                                    : (static_cast<size_t>(bhkv) * p.N + (key_live ? key : 0)) * HD;
       __nv_bfloat16* out = (half == 0 ? p.dv : p.dk) + row_off;
       float* acc = p.head_split > 1 ? (half == 0 ? p.dv_acc : p.dk_acc) + row_off : nullptr;
       const uint32_t col = half == 0 ? C::T_DV : C::T_DK;
@@ -464,7 +543,9 @@ __global__ void __launch_bounds__(512, 1)
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (tid == 0 && ok) {
-          tma_reduce_add_3d(&tm_dq, sDQ, c * 32, q0, bhq);
+          int qy, qz;
+          q_yz(bhq, q0, qy, qz);
+          tma_reduce_add_3d(&tm_dq, sDQ, c * 32, qy, qz);
           bulk_commit_group();
         }
       }

@@ -67,6 +67,79 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdPrepParams p)
   }
 }
 
+// First workspace row of sequence s in the variable-length backward:
+// 4 ceil(cu_q[s] / 4) + 4 s. Multiples of 4 (16 bytes of f32), and each
+// sequence's rows end before the next one's start (the gap covers the round
+// up); a head's row holds ws_seq_base(total_q, batch) + 128 floats, so the
+// last sequence's 128-row tiles stay inside it.
+FA_DEV int ws_seq_base(int cu_q_s, int s) { return ((cu_q_s + 3) & ~3) + 4 * s; }
+
+struct BwdPrepVarlenParams {
+  const __nv_bfloat16* o;   // [total_q][Hq][d]
+  const __nv_bfloat16* dO;
+  const float* lse;         // [total_q][Hq]
+  float* ws_delta;          // [Hq][Npad]
+  float* ws_lse2;           // [Hq][Npad]
+  float* dq_acc;            // [total_q][Hq][d]
+  const int* cu_q;
+  int batch, Hq, Npad, total_q;
+};
+
+// Variable-length preprocess: every workspace row of every head is written,
+// a row inside a sequence with D and LSE * log2(e) (and its dQ accumulator
+// row zeroed), a row of the padding between sequences with 0 and +inf. The
+// sequence of a row is found by bisection over the (monotone) sequence bases.
+// 8 threads per row, 32 rows per block; grid (Npad / 32) * Hq.
+template <int HD>
+__global__ void __launch_bounds__(256) fa_bwd_prep_varlen_kernel(const BwdPrepVarlenParams p) {
+  constexpr int PER = HD / 8;
+  const int blocks_per_head = p.Npad / 32;
+  const int h = static_cast<int>(blockIdx.x) / blocks_per_head;
+  const int sub = threadIdx.x & 7;
+  const int w = (static_cast<int>(blockIdx.x) - h * blocks_per_head) * 32 + (threadIdx.x >> 3);
+  // largest s with ws_seq_base(cu_q[s], s) <= w (base of sequence 0 is 0)
+  int lo = 0, hi = p.batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ws_seq_base(__ldg(p.cu_q + mid), mid) <= w) lo = mid;
+    else hi = mid - 1;
+  }
+  const int tok0 = __ldg(p.cu_q + lo);
+  const int i = w - ws_seq_base(tok0, lo);
+  // (offsets that break the sizes are reported by the main kernel; here they
+  // only must not lead outside the tensors)
+  const bool live = i < __ldg(p.cu_q + lo + 1) - tok0 && tok0 >= 0 && tok0 + i < p.total_q;
+  const size_t row = static_cast<size_t>(tok0 + (live ? i : 0)) * p.Hq + h;
+  float acc = 0.f;
+  if (live) {
+    const size_t off = row * HD + sub * PER;
+    const uint4* o4 = reinterpret_cast<const uint4*>(p.o + off);
+    const uint4* d4 = reinterpret_cast<const uint4*>(p.dO + off);
+    float4* z4 = reinterpret_cast<float4*>(p.dq_acc + off);
+#pragma unroll
+    for (int j = 0; j < PER / 8; ++j) {
+      const uint4 a = o4[j], g = d4[j];
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        acc = fmaf(bf16_lo(av[t]), bf16_lo(gv[t]), acc);
+        acc = fmaf(bf16_hi(av[t]), bf16_hi(gv[t]), acc);
+      }
+      z4[2 * j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z4[2 * j + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+  if (sub == 0) {
+    const size_t wi = static_cast<size_t>(h) * p.Npad + w;
+    p.ws_delta[wi] = live ? acc : 0.f;
+    p.ws_lse2[wi] = live ? p.lse[row] * 1.4426950408889634f : INFINITY;
+  }
+}
+
 // ------------------------------------------------------------ dQ convert
 
 // grid-stride over float4 groups of the accumulator: dq = bf16(acc).

@@ -106,6 +106,8 @@ int prepare_kernels(int dev) {
   set_decode_attributes<256>(set);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64>), fa::Bwd2Cfg<64>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128>), fa::Bwd2Cfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64, true>), fa::Bwd2Cfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128, true>), fa::Bwd2Cfg<128>::SMEM_BYTES);
   if (e != cudaSuccess) return FA_ERR_CUDA;
   done[dev] = true;
   return FA_OK;
@@ -523,6 +525,117 @@ int launch_bwd_stages(const BwdPlan& pl, unsigned stages) {
   return FA_OK;
 }
 
+// ------------------------------------------------- variable-length backward
+//
+// Workspace, all f32: D and LSE * log2(e) [Hq][Npad] with Npad covering every
+// sequence's rows from ws_seq_base(cu_q[s], s) plus a 128-row tail; the dQ
+// accumulator [total_q][Hq][d]; with a head split, dK and dV accumulators
+// [total_k][Hkv][d]. The split estimate counts the key tiles of total_k.
+size_t bwd_varlen_npad(int batch, int total_q) {
+  const size_t rows = ((static_cast<size_t>(total_q) + 3) & ~static_cast<size_t>(3)) + 4 * static_cast<size_t>(batch) + 128;
+  return (rows + 127) / 128 * 128;
+}
+
+int bwd_varlen_head_split(int total_k, int Hq, int Hkv) { return bwd_head_split(1, Hq, Hkv, total_k); }
+
+size_t bwd_varlen_workspace_bytes(int batch, int total_q, int total_k, int Hq, int Hkv, int d) {
+  const size_t kv_acc =
+      bwd_varlen_head_split(total_k, Hq, Hkv) > 1 ? 2 * static_cast<size_t>(total_k) * Hkv * d : 0;
+  return sizeof(float) * (2 * static_cast<size_t>(Hq) * bwd_varlen_npad(batch, total_q) +
+                          static_cast<size_t>(total_q) * Hq * d + kv_acc);
+}
+
+template <int HD>
+int run_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                   void* dq, void* dk, void* dv, const int* cu_q, const int* cu_k, int batch, int max_seqlen_q,
+                   int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, float scale, int causal, void* ws,
+                   cudaStream_t stream) {
+  using C = fa::Bwd2Cfg<HD>;
+  // plan everything before the first launch
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD, true>)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (attr.numRegs != C::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;  // the register split needs exactly this
+  const size_t npad = bwd_varlen_npad(batch, total_q);
+  const int split = bwd_varlen_head_split(total_k, Hq, Hkv);
+  const size_t q_elems = static_cast<size_t>(total_q) * Hq * HD;
+  const size_t kv_elems = static_cast<size_t>(total_k) * Hkv * HD;
+  float* delta = static_cast<float*>(ws);
+  float* lse2 = delta + static_cast<size_t>(Hq) * npad;
+  float* dq_acc = lse2 + static_cast<size_t>(Hq) * npad;
+  float* dk_acc = split > 1 ? dq_acc + q_elems : nullptr;
+  float* dv_acc = split > 1 ? dk_acc + kv_elems : nullptr;
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  int rc = make_map3(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hq, total_q, 64, 1, 128);
+  if (rc == FA_OK) rc = make_map3(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hkv, total_k, 64, 1, 128);
+  if (rc == FA_OK) rc = make_map3(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hkv, total_k, 64, 1, 128);
+  if (rc == FA_OK) rc = make_map3(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hq, total_q, 64, 1, 128);
+  if (rc == FA_OK) rc = make_map3(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, Hq, total_q, 32, 1, 128);
+  if (rc != FA_OK) return rc;
+  fa::BwdPrepVarlenParams pp;
+  pp.o = static_cast<const __nv_bfloat16*>(o);
+  pp.dO = static_cast<const __nv_bfloat16*>(dO);
+  pp.lse = lse;
+  pp.ws_delta = delta;
+  pp.ws_lse2 = lse2;
+  pp.dq_acc = dq_acc;
+  pp.cu_q = cu_q;
+  pp.batch = batch;
+  pp.Hq = Hq;
+  pp.Npad = static_cast<int>(npad);
+  pp.total_q = total_q;
+  const long long prep_blocks = static_cast<long long>(npad / 32) * Hq;
+  fa::Bwd2Params mp{};
+  mp.ws_delta = delta;
+  mp.ws_lse2 = lse2;
+  mp.dq_acc = dq_acc;
+  mp.dk = static_cast<__nv_bfloat16*>(dk);
+  mp.dv = static_cast<__nv_bfloat16*>(dv);
+  mp.dk_acc = dk_acc;
+  mp.dv_acc = dv_acc;
+  mp.head_split = split;
+  mp.BHkv = batch * Hkv;
+  mp.N = 0;
+  mp.Npad = static_cast<int>(npad);
+  mp.Hq = Hq;
+  mp.Hkv = Hkv;
+  mp.num_tiles = (max_seqlen_k + 127) / 128;
+  mp.scale_log2 = scale * 1.4426950408889634f;
+  mp.scale = scale;
+  mp.causal = causal;
+  mp.timeout_ns = timeout_now();
+  mp.cu_q = cu_q;
+  mp.cu_k = cu_k;
+  mp.batch = batch;
+  mp.total_q = total_q;
+  mp.total_k = total_k;
+  mp.max_seqlen_q = max_seqlen_q;
+  mp.max_seqlen_k = max_seqlen_k;
+  const long long main_blocks = static_cast<long long>(mp.num_tiles) * batch * Hkv * split;
+  if (prep_blocks > INT32_MAX || main_blocks > INT32_MAX || npad > static_cast<size_t>(INT32_MAX))
+    return FA_ERR_INVALID;
+  // launches
+  fa::fa_bwd_prep_varlen_kernel<HD><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(pp);
+  if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  if (split > 1) {  // zero the f32 dK and dV accumulators (contiguous)
+    fa::fa_zero_f32_kernel<<<grid_stride_blocks(kv_elems / 2), 256, 0, stream>>>(dk_acc, kv_elems / 2);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  fa::fa_bwd2_main_kernel<HD, true><<<static_cast<unsigned>(main_blocks), C::THREADS, C::SMEM_BYTES, stream>>>(
+      mq, mk, mv, mdo, mdq, mp);
+  if (launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD, true>)) != FA_OK) return FA_ERR_CUDA;
+  if (split > 1) {
+    fa::fa_bwd_dq_kernel<<<grid_stride_blocks(kv_elems / 4), 256, 0, stream>>>(dk_acc, mp.dk, kv_elems / 4);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+    fa::fa_bwd_dq_kernel<<<grid_stride_blocks(kv_elems / 4), 256, 0, stream>>>(dv_acc, mp.dv, kv_elems / 4);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  fa::fa_bwd_dq_kernel<<<grid_stride_blocks(q_elems / 4), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
+                                                                           q_elems / 4);
+  if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 // KV-cache forward: R query rows per KV head, S key splits of L keys (L a
 // multiple of 64). About four CTAs per SM of a 148-SM part, at least 256 keys
 // per split; a pure function of the sizes.
@@ -754,6 +867,59 @@ int fa_merge_partials(const void* o_parts, const float* lse_parts, int n_parts, 
     case 128: return launch_merge<128>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
     default: return launch_merge<256>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
   }
+}
+
+size_t fa_bwd_varlen_workspace_size(int batch, int total_q, int total_k, int Hq, int Hkv, int d) {
+  if (batch < 0 || total_q < 0 || total_k < 0 || Hq < 1 || Hkv < 1 || d < 1 || Hq % Hkv != 0) return 0;
+  return bwd_varlen_workspace_bytes(batch, total_q, total_k, Hq, Hkv, d);
+}
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                  void* dq, void* dk, void* dv, const int* cu_seqlens_q, const int* cu_seqlens_k, int batch,
+                  int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, float scale,
+                  int causal, void* workspace, size_t workspace_bytes, int dtype, fa_stream_t stream) {
+  if (batch < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || total_q < 0 || total_k < 0 || Hq < 1 || Hkv < 1 ||
+      d < 1)
+    return FA_ERR_INVALID;
+  if (Hq % Hkv != 0 || (causal != 0 && causal != 1) || !std::isfinite(scale)) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if (batch == 0 || total_k == 0) return FA_OK;
+  if (total_q == 0) {
+    // no queries at all: every key's gradient is zero
+    if (!aligned16(dk) || !aligned16(dv)) return FA_ERR_INVALID;
+    int dev = 0;
+    int rc = check_device(&dev);
+    if (rc != FA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t n4 = static_cast<size_t>(total_k) * Hkv * d / 8;  // bf16 elements, 8 per 16 bytes
+    fa::fa_zero_f32_kernel<<<grid_stride_blocks(n4), 256, 0, s>>>(static_cast<float*>(dk), n4);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+    fa::fa_zero_f32_kernel<<<grid_stride_blocks(n4), 256, 0, s>>>(static_cast<float*>(dv), n4);
+    return launch_status();
+  }
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k || max_seqlen_k < 1 ||
+      static_cast<long long>(total_q) * Hq > INT32_MAX / 2 || static_cast<long long>(total_k) * Hkv > INT32_MAX / 2 ||
+      total_q > INT32_MAX - 4 * batch - 256)
+    return FA_ERR_INVALID;
+  for (const void* ptr : std::initializer_list<const void*>{q, k, v, o, lse, dO, dq, dk, dv})
+    if (!aligned16(ptr)) return FA_ERR_INVALID;
+  for (const int* cu : {cu_seqlens_q, cu_seqlens_k})
+    if (cu == nullptr || (reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return FA_ERR_INVALID;
+  if (workspace == nullptr || !aligned16(workspace) ||
+      workspace_bytes < bwd_varlen_workspace_bytes(batch, total_q, total_k, Hq, Hkv, d))
+    return FA_ERR_WORKSPACE;
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != FA_OK) return rc;
+  if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? run_bwd_varlen<64>(q, k, v, o, lse, dO, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, batch,
+                                      max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, scale, causal,
+                                      workspace, s)
+                 : run_bwd_varlen<128>(q, k, v, o, lse, dO, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, batch,
+                                       max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, scale, causal,
+                                       workspace, s);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {

@@ -68,7 +68,6 @@ struct Fwd2Params {
   int diag_shift;
 };
 
-constexpr int kStatusInvalid = 1;  // equals FA_ERR_INVALID: sequence offsets inconsistent with the sizes given
 
 // ---------------------------------------------------------------- helpers
 

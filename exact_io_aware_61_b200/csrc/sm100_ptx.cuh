@@ -18,6 +18,7 @@ __device__ int g_status;
 
 constexpr int kStatusTimeout = 4;  // equals FA_ERR_TIMEOUT
 constexpr int kStatusLayout = 2;   // equals FA_ERR_UNSUPPORTED: shared memory not laid out as the kernel needs
+constexpr int kStatusInvalid = 1;  // equals FA_ERR_INVALID: sequence offsets inconsistent with the sizes given
 
 FA_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -77,9 +77,11 @@ def as_f64(t: torch.Tensor):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def make_varlen_inputs(lens_q, lens_k, Hq: int, Hkv: int, d: int, dtype: str = "bf16", seed: int = 0):
+def make_varlen_inputs(lens_q, lens_k, Hq: int, Hkv: int, d: int, dtype: str = "bf16", seed: int = 0,
+                       grad: bool = False):
     """A packed batch of sequences: ``q [sum(lens_q), Hq, d]``, ``k, v [sum(lens_k), Hkv, d]`` (CPU) and
-    the int32 offsets ``cu_q``, ``cu_k`` (batch + 1 entries from 0). Same recipe as :func:`make_inputs`."""
+    the int32 offsets ``cu_q``, ``cu_k`` (batch + 1 entries from 0); with ``grad`` also an upstream
+    gradient ``do`` shaped like ``q``. Same recipe as :func:`make_inputs`."""
     if len(lens_q) != len(lens_k):
         raise ValueError("one query length and one key length per sequence")
     g = torch.Generator(device="cpu").manual_seed(int(seed))
@@ -89,6 +91,8 @@ def make_varlen_inputs(lens_q, lens_k, Hq: int, Hkv: int, d: int, dtype: str = "
         "k": torch.randn((tk, Hkv, d), generator=g, dtype=torch.float32),
         "v": torch.randn((tk, Hkv, d), generator=g, dtype=torch.float32),
     }
+    if grad:
+        out["do"] = torch.randn((tq, Hq, d), generator=g, dtype=torch.float32)
     if dtype == "bf16":
         out = {name: t.to(torch.bfloat16) for name, t in out.items()}
     cu = lambda lens: torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32)

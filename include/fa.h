@@ -286,6 +286,53 @@ FA_API int fa_bwd_noalloc(const void* q, const void* k, const void* v, const voi
                    int dtype, fa_stream_t stream);
 
 /*
+ * fa_bwd_varlen_workspace_size -- bytes of device workspace fa_bwd_varlen
+ * needs: 4 * (2 * Hq * P + total_q * Hq * d + A), where P = the multiple
+ * of 128 at or above 4 * ceil(total_q / 4) + 4 * batch + 128 (per query
+ * head, the D and LSE rows of every sequence, each starting on a 16-byte
+ * boundary, with a 128-row tail) and A = 2 * total_k * Hkv * d when the
+ * group's query heads are split over several CTAs per key tile (the same
+ * rule as fa_bwd_workspace_size with B = 1, N = total_k), else 0. A pure
+ * function of the sizes. Returns 0 for invalid sizes.
+ */
+FA_API size_t fa_bwd_varlen_workspace_size(int batch, int total_q, int total_k, int Hq,
+                                           int Hkv, int d);
+
+/*
+ * fa_bwd_varlen -- backward pass over a packed batch of sequences of
+ * different lengths (or strided BNHD tensors), the gradient of fa_fwd_varlen.
+ *
+ *   q, o, dO [total_q][Hq][d]        inputs (bf16); o and lse from
+ *   lse [total_q][Hq]                fa_fwd_varlen on the same q, k, v
+ *   k, v [total_k][Hkv][d]           inputs (bf16)
+ *   dq [total_q][Hq][d]              output (bf16)
+ *   dk, dv [total_k][Hkv][d]         outputs (bf16): dK, dV summed over the
+ *                                    query heads of each KV head's group
+ *   cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q, total_q, total_k:
+ *                                    as fa_fwd_varlen; max_seqlen_k the
+ *                                    longest key sequence
+ *   workspace                        device memory, at least
+ *                                    fa_bwd_varlen_workspace_size bytes,
+ *                                    16-byte aligned; overwritten
+ * Each sequence is its own problem with its queries at its last positions,
+ * as in the forward; the formulas are fa_bwd's ("The backward pass, and
+ * where the memory saving comes from": scores recomputed from Q and K, the
+ * weights rebuilt from the stored LSE). Keys that no query sees, and every
+ * key of a sequence with no queries, get zero gradients. dtype FA_BF16 with
+ * d in {64, 128}; other cases return FA_ERR_UNSUPPORTED. As in the forward,
+ * the offsets' consistency is checked on the device (FA_ERR_INVALID in the
+ * device status word; the sequence is skipped). dQ is accumulated with f32
+ * atomics, so its last bit may differ between runs. batch == 0 or
+ * total_k == 0 is a no-op. Returns fa_status.
+ */
+FA_API int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int batch,
+                  int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                  int Hq, int Hkv, int d, float scale, int causal, void* workspace,
+                  size_t workspace_bytes, int dtype, fa_stream_t stream);
+
+/*
  * fa_fwd_kvcache_workspace_size -- bytes of device workspace fa_fwd_kvcache
  * needs: per key split, the softmax state (max, sum, unnormalised output row)
  * of each of the R = (Hq / Hkv) * Nq query rows of a KV head, float32:
