@@ -24,6 +24,7 @@
 #include "fwd_f32.cuh"
 #include "bwd_sm100.cuh"
 #include "bwd2_sm100.cuh"
+#include "bwd256_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "merge_sm100.cuh"
 
@@ -108,6 +109,7 @@ int prepare_kernels(int dev) {
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128>), fa::Bwd2Cfg<128>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64, true>), fa::Bwd2Cfg<64>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128, true>), fa::Bwd2Cfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd256_main_kernel), fa::Bwd256Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return FA_ERR_CUDA;
   done[dev] = true;
   return FA_OK;
@@ -350,13 +352,16 @@ int launch_fwd_f32(const void* q, const void* k, const void* v, void* o, float* 
 
 size_t padded_rows(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 
-// How many CTAs share the query heads of one (KV head, 128-key tile) in the
+// How many CTAs share the query heads of one (KV head, key tile) in the
 // backward: 1 unless B * Hkv * (key tiles) is below 592 (4 CTAs per SM of a
 // 148-SM part), then the smallest divisor of the group size that reaches it,
-// or the group size. A pure function of the shape, so the workspace size
-// does not depend on the device.
-int bwd_head_split(int B, int Hq, int Hkv, int N) {
-  const long long ctas = static_cast<long long>(B) * Hkv * static_cast<long long>(padded_rows(N) / 128);
+// or the group size. Key tiles hold 128 keys (64 at d = 256). A pure function
+// of the shape, so the workspace size does not depend on the device.
+int bwd_key_tile(int d) { return d == 256 ? 64 : 128; }
+
+int bwd_head_split(int B, int Hq, int Hkv, int N, int d = 128) {
+  const int tile = bwd_key_tile(d);
+  const long long ctas = static_cast<long long>(B) * Hkv * ((static_cast<long long>(N) + tile - 1) / tile);
   const int g = Hq / Hkv;
   for (int s = 1; s <= g; ++s)
     if (g % s == 0 && ctas * s >= 592) return s;
@@ -376,7 +381,7 @@ struct BwdWorkspace {
 
 size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   const size_t rows_q = static_cast<size_t>(B) * Hq;
-  const size_t kv_acc = bwd_head_split(B, Hq, Hkv, N) > 1 ? 2 * static_cast<size_t>(B) * Hkv * N * d : 0;
+  const size_t kv_acc = bwd_head_split(B, Hq, Hkv, N, d) > 1 ? 2 * static_cast<size_t>(B) * Hkv * N * d : 0;
   return sizeof(float) * (2 * rows_q * padded_rows(N) + rows_q * static_cast<size_t>(N) * d + kv_acc);
 }
 
@@ -388,7 +393,7 @@ BwdWorkspace carve(void* ws, int B, int Hq, int Hkv, int N, int d) {
   w.delta = static_cast<float*>(ws);
   w.lse2 = w.delta + rows_q * npad;
   w.dq_acc = w.lse2 + rows_q * npad;
-  const bool split = bwd_head_split(B, Hq, Hkv, N) > 1;
+  const bool split = bwd_head_split(B, Hq, Hkv, N, d) > 1;
   w.dk_acc = split ? w.dq_acc + rows_q * static_cast<size_t>(N) * d : nullptr;
   w.dv_acc = split ? w.dk_acc + kv_elems : nullptr;
   return w;
@@ -412,6 +417,7 @@ struct BwdPlan {
   unsigned prep_blocks;
   CUtensorMap mq, mk, mv, mdo, mdq;
   fa::Bwd2Params mp;
+  fa::Bwd256Params mp256;
   unsigned main_blocks;
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
@@ -423,12 +429,12 @@ template <int HD>
 int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const void* v, const void* o,
              const float* lse, const void* dO, void* dq, void* dk, void* dv, void* ws, int B, int Hq, int Hkv,
              int N, float scale, int causal, cudaStream_t stream) {
-  using C = fa::Bwd2Cfg<HD>;
+  using C = fa::Bwd2Cfg<HD == 256 ? 128 : HD>;
   pl->stream = stream;
   pl->w = carve(ws, B, Hq, Hkv, N, HD);
   pl->kv_elems = static_cast<size_t>(B) * Hkv * static_cast<size_t>(N) * HD;
   pl->q_elems = static_cast<size_t>(B) * Hq * static_cast<size_t>(N) * HD;
-  pl->split = bwd_head_split(B, Hq, Hkv, N);
+  pl->split = bwd_head_split(B, Hq, Hkv, N, HD);
   pl->dq = static_cast<__nv_bfloat16*>(dq);
   pl->dk = static_cast<__nv_bfloat16*>(dk);
   pl->dv = static_cast<__nv_bfloat16*>(dv);
@@ -448,12 +454,42 @@ int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const v
     if (blocks > INT32_MAX) return FA_ERR_INVALID;
     pl->prep_blocks = static_cast<unsigned>(blocks);
   }
-  if (stages & 2u) {
+  if ((stages & 2u) && HD == 256) {
+    // 64-key tiles: K and V boxes of 64 rows, Q and dO boxes of 128
+    int rc = make_map(&pl->mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
+    if (rc == FA_OK) rc = make_map(&pl->mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 64);
+    if (rc == FA_OK) rc = make_map(&pl->mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 64);
+    if (rc == FA_OK) rc = make_map(&pl->mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
+    if (rc != FA_OK) return rc;
+    fa::Bwd256Params& mp = pl->mp256;
+    mp.ws_delta = pl->w.delta;
+    mp.ws_lse2 = pl->w.lse2;
+    mp.dq_acc = pl->w.dq_acc;
+    mp.dk = pl->dk;
+    mp.dv = pl->dv;
+    mp.dk_acc = pl->w.dk_acc;
+    mp.dv_acc = pl->w.dv_acc;
+    mp.N = N;
+    mp.Npad = static_cast<int>(npad);
+    mp.Hq = Hq;
+    mp.Hkv = Hkv;
+    mp.num_tiles = (N + fa::Bwd256Cfg::BK - 1) / fa::Bwd256Cfg::BK;
+    mp.head_split = pl->split;
+    mp.BHkv = B * Hkv;
+    mp.scale_log2 = scale * 1.4426950408889634f;
+    mp.scale = scale;
+    mp.causal = causal;
+    mp.timeout_ns = timeout_now();
+    const long long blocks = static_cast<long long>(mp.num_tiles) * B * Hkv * pl->split;
+    if (blocks > INT32_MAX) return FA_ERR_INVALID;
+    pl->main_blocks = static_cast<unsigned>(blocks);
+  } else if (stages & 2u) {
     // The kernel redistributes registers between warpgroups (setmaxnreg) on
     // the assumption of exactly LAUNCH_REGS per thread at launch; a build
     // with another count would wait for ever, so it is refused here.
     cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>)) != cudaSuccess)
+    if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD == 256 ? 128 : HD>)) !=
+        cudaSuccess)
       return FA_ERR_CUDA;
     if (attr.numRegs != C::LAUNCH_REGS) {
       if (verbose()) std::fprintf(stderr, "fa: backward built with %d registers, expected %d\n", attr.numRegs,
@@ -495,7 +531,7 @@ int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const v
 
 template <int HD>
 int launch_bwd_stages(const BwdPlan& pl, unsigned stages) {
-  using C = fa::Bwd2Cfg<HD>;
+  using C = fa::Bwd2Cfg<HD == 256 ? 128 : HD>;
   if (stages & 1u) {
     fa::fa_bwd_prep_kernel<HD><<<pl.prep_blocks, 256, 0, pl.stream>>>(pl.pp);
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
@@ -506,9 +542,15 @@ int launch_bwd_stages(const BwdPlan& pl, unsigned stages) {
                                                                                         pl.kv_elems / 2);
       if (launch_status() != FA_OK) return FA_ERR_CUDA;
     }
-    fa::fa_bwd2_main_kernel<HD><<<pl.main_blocks, C::THREADS, C::SMEM_BYTES, pl.stream>>>(pl.mq, pl.mk, pl.mv,
-                                                                                          pl.mdo, pl.mdq, pl.mp);
-    if (launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>)) != FA_OK) return FA_ERR_CUDA;
+    if constexpr (HD == 256) {
+      fa::fa_bwd256_main_kernel<<<pl.main_blocks, fa::Bwd256Cfg::THREADS, fa::Bwd256Cfg::SMEM_BYTES, pl.stream>>>(
+          pl.mq, pl.mk, pl.mv, pl.mdo, pl.mp256);
+      if (launch_status(reinterpret_cast<const void*>(&fa::fa_bwd256_main_kernel)) != FA_OK) return FA_ERR_CUDA;
+    } else {
+      fa::fa_bwd2_main_kernel<HD><<<pl.main_blocks, C::THREADS, C::SMEM_BYTES, pl.stream>>>(pl.mq, pl.mk, pl.mv,
+                                                                                            pl.mdo, pl.mdq, pl.mp);
+      if (launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD>)) != FA_OK) return FA_ERR_CUDA;
+    }
     if (pl.split > 1) {
       const size_t n4 = pl.kv_elems / 4;
       fa::fa_bwd_dq_kernel<<<grid_stride_blocks(n4), 256, 0, pl.stream>>>(pl.w.dk_acc, pl.dk, n4);
@@ -733,7 +775,7 @@ int check_bwd(std::initializer_list<const void*> ptrs, void* workspace, size_t w
               int Hkv, int N, int d, float scale, int causal, int dtype, int* dev) {
   int rc = check_shape(B, Hq, Hkv, N, d, scale, causal, dtype);
   if (rc != FA_OK) return rc;
-  if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return -1;  // empty: nothing to launch
   for (const void* p : ptrs)
     if (!aligned16(p)) return FA_ERR_INVALID;
@@ -949,6 +991,12 @@ int run_bwd(unsigned stages, std::initializer_list<const void*> ptrs, const void
       return rc;
     return launch_bwd_stages<64>(pl, stages);
   }
+  if (d == 256) {
+    if ((rc = plan_bwd<256>(&pl, stages, q, k, v, o, lse, dO, dq, dk, dv, ws, B, Hq, Hkv, N, scale, causal, s)) !=
+        FA_OK)
+      return rc;
+    return launch_bwd_stages<256>(pl, stages);
+  }
   if ((rc = plan_bwd<128>(&pl, stages, q, k, v, o, lse, dO, dq, dk, dv, ws, B, Hq, Hkv, N, scale, causal, s)) !=
       FA_OK)
     return rc;
@@ -1030,7 +1078,7 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    int dtype, fa_stream_t stream) {
   int rc = check_shape(B, Hq, Hkv, N, d, scale, causal, dtype);
   if (rc != FA_OK) return rc;
-  if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return FA_OK;
   if (bwd_workspace_bytes(B, Hq, Hkv, N, d) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
   int dev = 0;

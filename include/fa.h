@@ -184,10 +184,11 @@ FA_API int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, f
  * per-row term D = rowsum(dO * O) and the log2-scaled LSE, both float32 and
  * padded to a multiple of 128 rows per head, plus a float32 dQ accumulator
  * [B][Hq][N][d]: 4 * (2 * B * Hq * Npad + B * Hq * N * d) bytes, Npad = N
- * rounded up to 128. When B * Hkv * ceil(N / 128) < 592, the backward
- * splits each group's query heads over several CTAs (the smallest divisor s
- * of Hq / Hkv with that product times s >= 592, else Hq / Hkv) and the
- * workspace also holds float32 dK and dV accumulators [B][Hkv][N][d].
+ * rounded up to 128. When B * Hkv * ceil(N / T) < 592, with key tiles of
+ * T = 128 keys (64 at d = 256), the backward splits each group's query
+ * heads over several CTAs (the smallest divisor s of Hq / Hkv with that
+ * product times s >= 592, else Hq / Hkv) and the workspace also holds
+ * float32 dK and dV accumulators [B][Hkv][N][d].
  * Linear in N: nothing N x N is ever allocated. Returns 0 for invalid sizes.
  */
 FA_API size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
@@ -207,11 +208,11 @@ FA_API size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
  * Recomputes every score tile from Q and K and the stored LSE ("The backward
  * pass, and where the memory saving comes from"): P = exp(scale*S - LSE),
  * dV = P^T dO, dP = dO V^T, dS = P * (dP - D), dQ = scale dS K,
- * dK = scale dS^T Q. Supports dtype FA_BF16 with d in {64, 128}; other
- * combinations return FA_ERR_UNSUPPORTED. Three kernels run in stream order:
+ * dK = scale dS^T Q. Supports dtype FA_BF16 with d in {64, 128, 256};
+ * FA_F32 returns FA_ERR_UNSUPPORTED. Three kernels run in stream order:
  * D and LSE preparation (and zeroing of the dQ accumulator), the main
- * recompute kernel (one CTA per 128-key tile: dK and dV, and each dQ tile
- * added into the f32 accumulator), and the dQ conversion; with split query
+ * recompute kernel (one CTA per 128-key tile, 64-key at d = 256: dK and dV,
+ * and each dQ tile added into the f32 accumulator), and the dQ conversion; with split query
  * heads (see fa_bwd_workspace_size) the main stage also zeroes the dK/dV
  * accumulators before, and rounds them to dk, dv after, its kernel. dq is
  * summed in whatever order the key tiles finish, so it can differ in the

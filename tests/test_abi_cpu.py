@@ -47,11 +47,12 @@ def test_status_strings(lib):
     assert "unknown" in fa.status_string(99)
 
 
-def _head_split(B, Hq, Hkv, N):
+def _head_split(B, Hq, Hkv, N, d=128):
     """CTAs per (KV head, key tile) in the backward: 1 when B*Hkv*tiles >= 592,
     else the smallest divisor of the group size that reaches 592, else the
-    group size."""
-    ctas = B * Hkv * ((N + 127) // 128)
+    group size. Key tiles of 128 keys, 64 at d = 256."""
+    tile = 64 if d == 256 else 128
+    ctas = B * Hkv * ((N + tile - 1) // tile)
     g = Hq // Hkv
     return next((s for s in range(1, g + 1) if g % s == 0 and ctas * s >= 592), g)
 
@@ -68,6 +69,11 @@ def test_workspace_formula(lib):
     # the split rule on a few shapes: MQA at 16k tokens, GQA at 16k (no split)
     assert _head_split(1, 32, 1, 16384) == 8
     assert _head_split(1, 32, 8, 16384) == 1
+    # d = 256 counts 64-key tiles: 1 x 4 KV heads x 74 tiles x 2 >= 592 (37 tiles x 4 at d = 128)
+    assert _head_split(1, 16, 4, 4736, 256) == 2 and _head_split(1, 16, 4, 4736, 128) == 4
+    assert fa.fa_bwd_workspace_size(1, 16, 4, 4736, 256) == 4 * (2 * 16 * 4736 + 16 * 4736 * 256 +
+                                                               2 * 4 * 4736 * 256)
+    assert fa.fa_bwd_workspace_size(2, 32, 32, 8192, 256) == 4 * (2 * 64 * 8192 + 64 * 8192 * 256)
     for shape in ((1, 32, 1, 16384, 128), (1, 32, 8, 16384, 128), (1, 8, 2, 4096, 128), (3, 6, 3, 700, 64)):
         B, Hq, Hkv, N, d = shape
         kv = 2 * B * Hkv * N * d if _head_split(B, Hq, Hkv, N) > 1 else 0
@@ -104,11 +110,11 @@ def test_validation_before_any_device_work(lib):
     # misaligned pointer
     p, m = ctypes.c_void_p(64), ctypes.c_void_p(66)
     assert lib.fa_fwd(p, p, m, p, p, 1, 1, 1, 8, 64, 0.1, 0, 0, None) == fa.FA_ERR_INVALID
-    # backward: f32 and d=256 are not implemented; short workspace
+    # backward: f32 is not implemented; short workspace (d = 256 included)
     p = ctypes.c_void_p(64)
     args = [p] * 9
     assert lib.fa_bwd(*args, p, 1 << 30, 1, 1, 1, 8, 64, 0.1, 0, 1, None) == fa.FA_ERR_UNSUPPORTED
-    assert lib.fa_bwd(*args, p, 1 << 30, 1, 1, 1, 8, 256, 0.1, 0, 0, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_bwd(*args, p, 16, 1, 1, 1, 8, 256, 0.1, 0, 0, None) == fa.FA_ERR_WORKSPACE
     assert lib.fa_bwd(*args, p, 16, 1, 1, 1, 8, 64, 0.1, 0, 0, None) == fa.FA_ERR_WORKSPACE
     assert lib.fa_bwd(*args, None, 1 << 30, 1, 1, 1, 8, 64, 0.1, 0, 0, None) == fa.FA_ERR_WORKSPACE
     assert lib.fa_selftest_wait_timeout(0, None) == fa.FA_ERR_INVALID
