@@ -448,8 +448,10 @@ def run_ours(args, rank, world, local):
     nbytes = algorithmic_bytes(B, Hq, Hkv, N, d)
     kf = kernel_flops(B, Hq, N, d, CAUSAL)
     src_hash = kernel_source_hash()
-    names = {"fwd": f"fa_fwd_bf16_2tile_kernel<{d}>", "bwd_prep": f"fa_bwd_prep_kernel<{d}>",
-             "bwd_main": f"fa_bwd2_main_kernel<{d}>", "bwd_dq": "fa_bwd_dq_kernel"}
+    names = {"fwd": f"fa_fwd_bf16_2tile_kernel<{d}>" if d != 256 else "fa_fwd_bf16_kernel<256>",
+             "bwd_prep": f"fa_bwd_prep_kernel<{d}>",
+             "bwd_main": f"fa_bwd2_main_kernel<{d}>" if d != 256 else "fa_bwd256_main_kernel",
+             "bwd_dq": "fa_bwd_dq_kernel"}
     kernels = {}
     for name, ms in per_kernel.items():
         e = {"kernel": names[name], "ms": round(ms, 4), "gbs": round(nbytes[name] / ms / 1e6, 1)}

@@ -29,11 +29,11 @@
 //               into 128-byte-swizzled shared tiles [query][key], which are
 //               the B operands of dV^T and dK^T and the A operand of dQ
 //   warps 8-11  dQ drain: thread = query row; loads a 128-column half of dQ
-//               from TMEM, frees it, adds it into the f32 accumulator
+//               from TMEM, frees it, then adds it into the f32 accumulator
 //               (red.global.add.v4.f32)
 //   warp 12     TMA producer; warp 13 TMEM allocator and MMA issuer
 // Per step (query tile t) the issuer runs S, dP, dV^T (once P is in shared
-// memory), dK^T (once dS is), dQ half 0, dQ half 1.
+// memory), dK^T (once dS is), dQ half 1, dQ half 0.
 #pragma once
 
 #include <cuda.h>
@@ -54,6 +54,15 @@ struct Bwd256Cfg {
   static constexpr int PS_BYTES = BQ * BK * 2;   // 16 KB: [128 q][64 keys], one 128-byte row per query
   static constexpr int SMEM_BYTES = 1024 + 2 * KV_BYTES + 2 * Q_BYTES + STATS_BYTES + 2 * PS_BYTES;
   static constexpr int THREADS = 512;
+  // Launch with 128 registers per thread (16 warps, 4 per SM sub-partition),
+  // then redistribute per warpgroup: the drain holds a whole 128-column half
+  // of the dQ tile, so that its columns are freed before any reduction.
+  static constexpr int LAUNCH_REGS = 128;
+  static constexpr int COMPUTE_REGS = 136;
+  static constexpr int DRAIN_REGS = 144;
+  static constexpr int OTHER_REGS = 96;
+  static_assert(128 * (2 * COMPUTE_REGS + DRAIN_REGS + OTHER_REGS) <= THREADS * LAUNCH_REGS,
+                "register split exceeds the launch allocation");
   static constexpr int KV_GROUP = 8;             // (batch, KV head) pairs scheduled together
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_DV = 0, T_DK = 128, T_S = 256, T_DP = 320, T_DQ0 = 384, T_DQ1 = 256;
@@ -75,8 +84,7 @@ struct Bwd256Params {
   unsigned long long timeout_ns;
 };
 
-// 16 warps, 4 per SM sub-partition: 128 registers each at launch (no
-// redistribution: the drain reads its dQ half in two 64-column pieces).
+// 16 warps, 4 per SM sub-partition: 16384 / 128 -> 128 registers at launch.
 __global__ void __launch_bounds__(512, 1)
     fa_bwd256_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -160,7 +168,9 @@ __global__ void __launch_bounds__(512, 1)
     bhq = b * p.Hq + hkv * group + h_first + hh;
   };
 
-  if (warp == 12) {
+  if (warp >= 12) {
+    set_max_regs<C::OTHER_REGS, C::LAUNCH_REGS>();
+    if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -193,7 +203,7 @@ __global__ void __launch_bounds__(512, 1)
       if (q_issued > 0) (void)mbar_wait_drain(smem_u32(&bar_qfull), (q_issued - 1) & 1, p.timeout_ns);
       if (do_issued > 0) (void)mbar_wait_drain(smem_u32(&bar_dofull), (do_issued - 1) & 1, p.timeout_ns);
     }
-  } else if (warp == 13) {
+    } else if (warp == 13) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);   // S, dP: [q x keys]
@@ -241,26 +251,31 @@ __global__ void __launch_bounds__(512, 1)
             mma_bf16_ss(tmem + C::T_DK + h * 64, sdesc_sw128(sQ + 2 * h * C::Q_CHUNK + kk * 2048, C::Q_CHUNK, 1024),
                         sdesc_sw128(sDS + kk * 2048, 8192, 1024), id_t, t > 0 || kk > 0);
         mma_commit(smem_u32(&bar_qempty));
-        // dQ = dS K, half 0 into its own columns, half 1 over S and dP (both
-        // read by the compute warps before they formed dS)
-        if (t > 0 && !mbar_wait(smem_u32(&bar_dq0free), ph ^ 1, wc)) { ok = false; break; }
+        // dQ = dS K in two 128-column halves: half 1 first, over S and dP
+        // (both read by the compute warps before they formed dS), so the
+        // drain frees those columns, which S(t+1) needs, as early as it can;
+        // half 0 into its own columns once the drain has read half 0 of dQ(t-1)
         tc_fence_after();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int i = 0; i < 2; ++i) {
+          const int h = 1 - i;
+          if (h == 0 && t > 0 && !mbar_wait(smem_u32(&bar_dq0free), ph ^ 1, wc)) { ok = false; break; }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_ss(tmem + (h == 0 ? C::T_DQ0 : C::T_DQ1), sdesc_sw128(sDS + kk * 32, 16, 1024),
                         sdesc_sw128(sK + 2 * h * C::KV_CHUNK + kk * 2048, C::KV_CHUNK, 1024), id_q, kk > 0);
           mma_commit(smem_u32(h == 0 ? &bar_dq0full : &bar_dq1full));
         }
+        if (!ok) break;
         mma_commit(smem_u32(&bar_dsempty));
       }
       // no MMA may be in flight when tensor memory is released
       mma_commit(smem_u32(&bar_final));
       (void)mbar_wait_drain(smem_u32(&bar_final), 0, p.timeout_ns);
     }
-  }
-  else if (warp < 8) {
+    }  // warps 14, 15: idle
+  } else if (warp < 8) {
+    set_max_regs<C::COMPUTE_REGS, C::LAUNCH_REGS>();
     // ---------------------------------------------------- compute warpgroups
     // Thread = query row r of the step's tile (TMEM lane r); warpgroup h
     // owns key columns [32h, 32h + 32), i.e. 16-byte chunks 4h .. 4h + 3 of
@@ -351,11 +366,12 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-  } else if (warp < 12) {
+  } else {
+    set_max_regs<C::DRAIN_REGS, C::LAUNCH_REGS>();
     // ------------------------------------------------------------ dQ drain
-    // Thread = query row r; each half of dQ is read in two 64-column pieces,
-    // its columns freed after the second, and added into the f32
-    // accumulator with 16-byte reductions.
+    // Thread = query row r. Per half (half 1 first, in the order the MMAs
+    // produce them): the whole 128-column half is loaded, its columns freed,
+    // then added into the f32 accumulator with 16-byte reductions.
     const int r = threadIdx.x - 256;
     const uint32_t lane_base = ((warp & 3) * 32u) << 16;
     bool ok = true;
@@ -365,35 +381,33 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t ph = t & 1;
       const bool live = q0 + r < p.N;
       float* row = p.dq_acc + (static_cast<size_t>(bhq) * p.N + (live ? q0 + r : 0)) * C::HD;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+#pragma unroll 1
+      for (int i = 0; i < 2; ++i) {
+        const int half = 1 - i;
         if (!warp_wait(smem_u32(half == 0 ? &bar_dq0full : &bar_dq1full), ph, wc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t src = tmem + lane_base + (half == 0 ? C::T_DQ0 : C::T_DQ1);
+        uint32_t v[4][32];
 #pragma unroll
-        for (int piece = 0; piece < 2; ++piece) {
-          uint32_t a[32], bb[32];
-          tmem_ld32(src + piece * 64, a);
-          tmem_ld32(src + piece * 64 + 32, bb);
-          if (piece == 1) {
-            tc_fence_before();
-            mbar_arrive(smem_u32(half == 0 ? &bar_dq0free : &bar_dq1free));
-          }
-          if (live) {
-            float* dst = row + half * 128 + piece * 64;
+        for (int c = 0; c < 4; ++c) tmem_ld32_async(src + c * 32, v[c]);
+        tmem_wait_ld32(v[0]);
 #pragma unroll
-            for (int x = 0; x < 8; ++x)
-              red_add_v4_f32(dst + 4 * x, __uint_as_float(a[4 * x]), __uint_as_float(a[4 * x + 1]),
-                             __uint_as_float(a[4 * x + 2]), __uint_as_float(a[4 * x + 3]));
+        for (int c = 1; c < 4; ++c) tmem_tie32(v[c]);
+        tc_fence_before();
+        mbar_arrive(smem_u32(half == 0 ? &bar_dq0free : &bar_dq1free));
+        if (live) {
+          float* dst = row + half * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int x = 0; x < 8; ++x)
-              red_add_v4_f32(dst + 32 + 4 * x, __uint_as_float(bb[4 * x]), __uint_as_float(bb[4 * x + 1]),
-                             __uint_as_float(bb[4 * x + 2]), __uint_as_float(bb[4 * x + 3]));
-          }
+              red_add_v4_f32(dst + c * 32 + 4 * x, __uint_as_float(v[c][4 * x]), __uint_as_float(v[c][4 * x + 1]),
+                             __uint_as_float(v[c][4 * x + 2]), __uint_as_float(v[c][4 * x + 3]));
         }
       }
     }
   }
+
   // warps 14, 15: idle
 
   tc_fence_before();

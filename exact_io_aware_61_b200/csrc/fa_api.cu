@@ -455,6 +455,12 @@ int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const v
     pl->prep_blocks = static_cast<unsigned>(blocks);
   }
   if ((stages & 2u) && HD == 256) {
+    // the kernel redistributes registers between warpgroups (setmaxnreg)
+    // assuming exactly LAUNCH_REGS per thread at launch: refuse another count
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_bwd256_main_kernel)) != cudaSuccess)
+      return FA_ERR_CUDA;
+    if (attr.numRegs != fa::Bwd256Cfg::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
     // 64-key tiles: K and V boxes of 64 rows, Q and dO boxes of 128
     int rc = make_map(&pl->mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
     if (rc == FA_OK) rc = make_map(&pl->mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 64);
