@@ -99,11 +99,11 @@ int prepare_kernels(int dev) {
   set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<64, true>), fa::Fwd2Cfg<64>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<128, true>), fa::Fwd2Cfg<128>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<256>), fa::FwdCfg<256>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<64, true>), fa::FwdCfg<64, true>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<128, true>), fa::FwdCfg<128, true>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<64>), fa::fwd_f32_smem_bytes<64>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<128>), fa::fwd_f32_smem_bytes<128>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<256>), fa::fwd_f32_smem_bytes<256>());
-  set_decode_attributes<64>(set);
-  set_decode_attributes<128>(set);
   set_decode_attributes<256>(set);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64>), fa::Bwd2Cfg<64>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128>), fa::Bwd2Cfg<128>::SMEM_BYTES);
@@ -710,13 +710,95 @@ int check_kvcache_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, float sca
   if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_INVALID;
   if (static_cast<long long>(B) * Hq > INT32_MAX / 2 || Nk > INT32_MAX - 256) return FA_ERR_INVALID;
   if (dtype != FA_BF16 || (d != 64 && d != 128 && d != 256)) return FA_ERR_UNSUPPORTED;
-  if (static_cast<long long>(Hq / Hkv) * Nq > 64) return FA_ERR_UNSUPPORTED;
+  // query rows per KV head: one 128-row MMA tile on the tensor cores (d = 64,
+  // 128), at most 64 rows in the d = 256 kernel
+  if (static_cast<long long>(Hq / Hkv) * Nq > (d == 256 ? 64 : 128)) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
+// KV-cache forward on the tensor cores (d = 64, 128): one CTA per (batch,
+// KV head, key split), one CTA per SM (its K/V ring fills shared memory and
+// it allocates all of TMEM). The split count minimises the estimated time,
+// waves x (tiles per split + a fixed cost of about two tiles per CTA); a
+// pure function of the sizes.
+struct DecodeTcPlan {
+  int S, split_tiles;
+};
+
+DecodeTcPlan decode_tc_plan(int B, int Hkv, int Nk) {
+  const long long pairs = static_cast<long long>(B) * Hkv;
+  const int tiles = (Nk + 127) / 128;
+  DecodeTcPlan best{1, tiles};
+  double best_cost = 1e300;
+  for (int s = 1; s <= std::min(tiles, 128); ++s) {
+    const int per = (tiles + s - 1) / s;
+    const int used = (tiles + per - 1) / per;  // splits actually needed at that size
+    const double waves = static_cast<double>((pairs * used + 147) / 148);
+    const double cost = waves * (per + 2.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = DecodeTcPlan{used, per};
+    }
+  }
+  return best;
+}
+
+bool decode_on_tensor_cores(int d) { return d == 64 || d == 128; }
+
 size_t kvcache_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  if (decode_on_tensor_cores(d)) {
+    // split parts of O (bf16) and LSE (f32) for the merge; none with one split
+    const DecodeTcPlan tp = decode_tc_plan(B, Hkv, Nk);
+    if (tp.S == 1) return 0;
+    return static_cast<size_t>(tp.S) * B * Hq * Nq * (2 * static_cast<size_t>(d) + 4);
+  }
   const DecodePlan dp = decode_plan(B, Hq, Hkv, Nq, Nk);
   return sizeof(float) * static_cast<size_t>(B) * Hkv * dp.S * dp.R * (static_cast<size_t>(d) + 2);
+}
+
+template <int HD>
+int launch_decode_tc(const void* q, const void* k, const void* v, void* o, float* lse, void* ws, int B, int Hq,
+                     int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream) {
+  using C = fa::FwdCfg<HD, true>;
+  const DecodeTcPlan tp = decode_tc_plan(B, Hkv, Nk);
+  const int R = (Hq / Hkv) * Nq;
+  const long long rows_total = static_cast<long long>(B) * Hq * Nq;
+  const long long blocks = static_cast<long long>(B) * Hkv * tp.S;
+  if (blocks > INT32_MAX || rows_total > INT32_MAX) return FA_ERR_INVALID;
+  CUtensorMap mq, mk, mv;
+  // Q as [B * Hq * Nq][d]: a KV head's R rows are contiguous
+  int rc = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, static_cast<uint64_t>(rows_total), 1, 64, 128);
+  if (rc == FA_OK) rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Nk, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  if (rc == FA_OK) rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Nk, static_cast<uint64_t>(B) * Hkv, 64, 128);
+  if (rc != FA_OK) return rc;
+  fa::FwdParams p{};
+  __nv_bfloat16* o_part = static_cast<__nv_bfloat16*>(o);
+  float* lse_part = lse;
+  if (tp.S > 1) {  // split parts in the workspace, merged below
+    o_part = static_cast<__nv_bfloat16*>(ws);
+    lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + static_cast<size_t>(tp.S) * rows_total * HD * 2);
+  }
+  p.o = o_part;
+  p.lse = lse_part;
+  p.N = Nk;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.timeout_ns = timeout_now();
+  p.R = R;
+  p.Nq = Nq;
+  p.splits = tp.S;
+  p.split_tiles = tp.split_tiles;
+  p.rows_total = static_cast<int>(rows_total);
+  fa::fa_fwd_bf16_kernel<HD, true><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  if (launch_status(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<HD, true>)) != FA_OK) return FA_ERR_CUDA;
+  if (tp.S == 1) return FA_OK;
+  int dev = 0, num_sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return launch_merge<HD>(o_part, lse_part, tp.S, rows_total, o, lse, num_sms, stream);
 }
 
 template <int HD, int RB>
@@ -1112,16 +1194,16 @@ int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* 
   if (B == 0) return FA_OK;
   for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(lse)})
     if (!aligned16(ptr)) return FA_ERR_INVALID;
-  if (workspace == nullptr || workspace_bytes < kvcache_workspace_bytes(B, Hq, Hkv, Nq, Nk, d))
-    return FA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return FA_ERR_INVALID;
+  const size_t need = kvcache_workspace_bytes(B, Hq, Hkv, Nq, Nk, d);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return FA_ERR_WORKSPACE;
+  if (need > 0 && !aligned16(workspace)) return FA_ERR_INVALID;
   int dev = 0;
   if ((rc = check_device(&dev)) != FA_OK) return rc;
   if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (d) {
-    case 64: return launch_decode_rows<64>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
-    case 128: return launch_decode_rows<128>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
+    case 64: return launch_decode_tc<64>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
+    case 128: return launch_decode_tc<128>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
     default: return launch_decode_rows<256>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
   }
 }

@@ -33,11 +33,13 @@
 
 namespace fa {
 
-template <int HD>
+// DECODE: the KV-cache configuration (one CTA per KV head and key split):
+// deeper K/V rings, since the whole CTA is a stream of K and V.
+template <int HD, bool DECODE = false>
 struct FwdCfg {
   static constexpr int BM = 128;  // query rows per CTA
   static constexpr int BN = 128;  // keys per tile
-  static constexpr int STAGES = HD == 64 ? 4 : (HD == 128 ? 2 : 1);
+  static constexpr int STAGES = DECODE ? (HD == 64 ? 6 : 3) : (HD == 64 ? 4 : (HD == 128 ? 2 : 1));
   static constexpr int Q_BYTES = BM * HD * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
   static constexpr int SMEM_BYTES = 1024 + Q_BYTES + 2 * STAGES * KV_BYTES;
@@ -57,13 +59,21 @@ struct FwdParams {
   // causal: query i sees key j iff j <= i + diag_shift; a row that sees no
   // key gets O = 0, LSE = -inf
   int diag_shift;
+  // DECODE kernel: N is the number of cached keys Nk; the R = (Hq / Hkv) * Nq
+  // query rows of KV head bh_kv are rows bh_kv * R .. bh_kv * R + R - 1 of Q
+  // viewed as [B * Hq * Nq][d] (query heads of a group, then queries), and row
+  // r is the query at position Nk - Nq + (r mod Nq). CTA (bh_kv, split s)
+  // takes key tiles [s * split_tiles, min((s + 1) * split_tiles, tiles)) and
+  // writes that split's normalised O and LSE to part s of o, lse laid out as
+  // [splits][rows_total = B * Hkv * R][d] and [splits][rows_total].
+  int R, Nq, splits, split_tiles, rows_total;
 };
 
-template <int HD>
+template <int HD, bool DECODE = false>
 __global__ void __launch_bounds__(192, 1)
     fa_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = FwdCfg<HD>;
+  using C = FwdCfg<HD, DECODE>;
   constexpr int ST = C::STAGES;
   constexpr int KCH = HD / 64;  // 64-column (128-byte) chunks per row
 
@@ -83,16 +93,29 @@ __global__ void __launch_bounds__(192, 1)
 
   // 1-D grid, head-major: consecutive CTAs share a KV head (its K/V tiles stay
   // in L2), and within a head the longest (last) query tiles start first.
-  const int bh = static_cast<int>(blockIdx.x) / p.num_q_tiles;
-  const int qt = p.num_q_tiles - 1 - (static_cast<int>(blockIdx.x) - bh * p.num_q_tiles);
-  const int b = bh / p.Hq;
-  const int hq = bh - b * p.Hq;
-  const int bh_kv = b * p.Hkv + hq / (p.Hq / p.Hkv);
-  const int q0 = qt * C::BM;
+  // DECODE: consecutive CTAs are the key splits of one KV head.
   const int n_kv_total = (p.N + C::BN - 1) / C::BN;
-  const int last_key = q0 + C::BM - 1 + p.diag_shift;  // causal: the last key any row of the tile sees
-  const int n_kv = !p.causal ? n_kv_total : last_key < 0 ? 0 : min(last_key / C::BN + 1, n_kv_total);
-  if (n_kv == 0) {
+  int bh, bh_kv, q0, n_kv, j0 = 0;
+  size_t out_base = 0;  // DECODE: first output row of this CTA
+  if constexpr (DECODE) {
+    bh_kv = static_cast<int>(blockIdx.x) / p.splits;
+    const int split = static_cast<int>(blockIdx.x) - bh_kv * p.splits;
+    j0 = split * p.split_tiles;
+    n_kv = min(n_kv_total, j0 + p.split_tiles) - j0;  // >= 1: the host sizes the splits
+    bh = bh_kv;
+    q0 = bh_kv * p.R;
+    out_base = static_cast<size_t>(split) * p.rows_total + static_cast<size_t>(bh_kv) * p.R;
+  } else {
+    bh = static_cast<int>(blockIdx.x) / p.num_q_tiles;
+    const int qt = p.num_q_tiles - 1 - (static_cast<int>(blockIdx.x) - bh * p.num_q_tiles);
+    const int b = bh / p.Hq;
+    const int hq = bh - b * p.Hq;
+    bh_kv = b * p.Hkv + hq / (p.Hq / p.Hkv);
+    q0 = qt * C::BM;
+    const int last_key = q0 + C::BM - 1 + p.diag_shift;  // causal: the last key any row of the tile sees
+    n_kv = !p.causal ? n_kv_total : last_key < 0 ? 0 : min(last_key / C::BN + 1, n_kv_total);
+  }
+  if (!DECODE && n_kv == 0) {
     // causal with a negative shift: no row of the tile sees a key
     const int row = q0 + threadIdx.x;
     if (threadIdx.x < C::BM && row < p.N) {
@@ -140,7 +163,7 @@ __global__ void __launch_bounds__(192, 1)
       prefetch_tmap(&tm_v);
       mbar_arrive_expect_tx(smem_u32(&bar_q), C::Q_BYTES);
       for (int c = 0; c < KCH; ++c)
-        tma_load_3d(sQ + c * (C::BM * 128), &tm_q, smem_u32(&bar_q), c * 64, q0, bh);
+        tma_load_3d(sQ + c * (C::BM * 128), &tm_q, smem_u32(&bar_q), c * 64, q0, DECODE ? 0 : bh);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % ST;
@@ -149,13 +172,13 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive_expect_tx(smem_u32(&bar_kfull[s]), C::KV_BYTES);
         for (int c = 0; c < KCH; ++c)
           tma_load_3d(sK + s * C::KV_BYTES + c * (C::BN * 128), &tm_k, smem_u32(&bar_kfull[s]), c * 64,
-                      j * C::BN, bh_kv);
+                      (j0 + j) * C::BN, bh_kv);
         k_issued = j + 1;
         if (!mbar_wait(smem_u32(&bar_vempty[s]), ph ^ 1, wc)) break;
         mbar_arrive_expect_tx(smem_u32(&bar_vfull[s]), C::KV_BYTES);
         for (int c = 0; c < KCH; ++c)
           tma_load_3d(sV + s * C::KV_BYTES + c * (C::BN * 128), &tm_v, smem_u32(&bar_vfull[s]), c * 64,
-                      j * C::BN, bh_kv);
+                      (j0 + j) * C::BN, bh_kv);
         v_issued = j + 1;
       }
       // leave no copy in flight into shared memory
@@ -212,6 +235,10 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------- softmax
     const int row = q0 + threadIdx.x;                 // this thread's query
     const uint32_t lane_base = (warp * 32u) << 16;    // TMEM lane field
+    // DECODE: the row's query sits at key position Nk - Nq + (r mod Nq); the
+    // causal limit of every row is at least Nk - Nq + 1 keys
+    const int dec_lim = !p.causal ? p.N : p.N - p.Nq + (DECODE ? static_cast<int>(threadIdx.x) % p.Nq : 0) + 1;
+    const int dec_first = !p.causal ? p.N : p.N - p.Nq + 1;
     float m_ref = -INFINITY;
     float l = 0.f;
     bool ok = true;
@@ -228,10 +255,11 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
       }
-      const int key0 = j * C::BN;
-      const bool diag = p.causal && (key0 + C::BN > q0 + p.diag_shift);
+      const int key0 = (j0 + j) * C::BN;
+      const bool diag = DECODE ? key0 + C::BN > dec_first : p.causal && (key0 + C::BN > q0 + p.diag_shift);
       if (diag || key0 + C::BN > p.N) {
-        const int lim = min(p.causal ? row + p.diag_shift + 1 : p.N, p.N) - key0;  // keys [key0, key0+lim) visible
+        // keys [key0, key0 + lim) visible
+        const int lim = (DECODE ? dec_lim : min(p.causal ? row + p.diag_shift + 1 : p.N, p.N)) - key0;
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= lim) s[c] = -INFINITY;
@@ -288,8 +316,9 @@ __global__ void __launch_bounds__(192, 1)
     if (ok && warp_wait(smem_u32(&bar_odone), (n_kv - 1) & 1, wc)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;  // l = 0: the row saw no key
-      const bool live = row < p.N;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (live ? row : 0)) * HD;
+      const bool live = DECODE ? static_cast<int>(threadIdx.x) < p.R : row < p.N;
+      const size_t o_row = DECODE ? out_base + (live ? threadIdx.x : 0) : static_cast<size_t>(bh) * p.N + (live ? row : 0);
+      __nv_bfloat16* orow = p.o + o_row * HD;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t r[32];
@@ -305,9 +334,7 @@ __global__ void __launch_bounds__(192, 1)
           for (int i = 0; i < 4; ++i) dst[i] = w[i];
         }
       }
-      if (live)
-        p.lse[static_cast<size_t>(bh) * p.N + row] =
-            l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      if (live) p.lse[o_row] = l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
   }
 

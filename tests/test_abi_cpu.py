@@ -129,13 +129,35 @@ def _decode_plan(B, Hq, Hkv, Nq, Nk):
     return (Hq // Hkv) * Nq, -(-Nk // L), L
 
 
+def _decode_tc_plan(B, Hkv, Nk):
+    """Key splits and 128-key tiles per split of the tensor-core KV-cache
+    forward (d = 64, 128): the smallest ceil(B*Hkv*S / 148) * (T + 2)."""
+    tiles = -(-Nk // 128)
+    best = None
+    for s in range(1, min(tiles, 128) + 1):
+        per = -(-tiles // s)
+        used = -(-tiles // per)
+        cost = -(-(B * Hkv * used) // 148) * (per + 2)
+        if best is None or cost < best[0]:
+            best = (cost, used, per)
+    return best[1], best[2]
+
+
 def test_kvcache_workspace_formula(lib):
-    for shape in ((1, 32, 8, 1, 32768, 128), (8, 32, 8, 1, 32768, 128), (2, 8, 2, 4, 1000, 64),
-                  (1, 2, 1, 16, 16, 256), (64, 16, 16, 1, 4096, 128)):
+    for shape in ((1, 2, 1, 16, 16, 256), (2, 8, 4, 2, 5000, 256)):
         B, Hq, Hkv, Nq, Nk, d = shape
         R, S, L = _decode_plan(B, Hq, Hkv, Nq, Nk)
         assert (S - 1) * L < Nk <= S * L and L % 64 == 0
         assert fa.fa_fwd_kvcache_workspace_size(*shape) == 4 * B * Hkv * S * R * (d + 2), shape
+    for shape in ((1, 32, 8, 1, 32768, 128), (8, 32, 8, 1, 32768, 128), (2, 8, 2, 4, 1000, 64),
+                  (64, 16, 16, 1, 4096, 128), (4, 32, 8, 4, 16384, 128), (1, 1, 1, 1, 100, 64)):
+        B, Hq, Hkv, Nq, Nk, d = shape
+        S, T = _decode_tc_plan(B, Hkv, Nk)
+        assert (S - 1) * T * 128 < Nk <= S * T * 128
+        want = 0 if S == 1 else S * B * Hq * Nq * (2 * d + 4)
+        assert fa.fa_fwd_kvcache_workspace_size(*shape) == want, shape
+    # MQA at 4k keys and batch 64: 2 splits of 16 tiles (128 CTAs, one wave)
+    assert _decode_tc_plan(64, 1, 4096) == (2, 16)
     assert fa.fa_fwd_kvcache_workspace_size(1, 2, 1, 9, 8, 64) == 0  # Nq > Nk
     assert fa.fa_fwd_kvcache_workspace_size(1, 3, 2, 1, 64, 64) == 0  # Hq not a multiple of Hkv
 
@@ -151,8 +173,9 @@ def test_kvcache_validation_before_any_device_work(lib):
     assert call(scale=float("nan")) == fa.FA_ERR_INVALID
     assert call(dtype=1) == fa.FA_ERR_UNSUPPORTED  # fp32
     assert call(d=96) == fa.FA_ERR_UNSUPPORTED
-    assert call(Hq=32, Hkv=1, Nq=3) == fa.FA_ERR_UNSUPPORTED  # 96 query rows per KV head > 64
-    assert call(ws_bytes=16) == fa.FA_ERR_WORKSPACE
+    assert call(Hq=32, Hkv=1, Nq=5) == fa.FA_ERR_UNSUPPORTED  # 160 query rows per KV head > 128
+    assert call(Hq=32, Hkv=1, Nq=3, d=256) == fa.FA_ERR_UNSUPPORTED  # 96 > 64 at d = 256
+    assert call(Nk=100000, ws_bytes=16) == fa.FA_ERR_WORKSPACE  # several key splits: parts to merge
     assert call(B=0) == fa.FA_OK  # empty problem
     m = ctypes.c_void_p(66)
     p = ctypes.c_void_p(64)

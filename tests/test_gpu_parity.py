@@ -404,6 +404,9 @@ KVCACHE_SHAPES = [  # (B, Hq, Hkv, Nq, Nk, d)
     (1, 2, 1, 16, 16, 128),    # Nq = Nk: the square problem
     (1, 16, 2, 8, 5000, 256),  # 64 rows per KV head at d = 256
     (2, 4, 1, 1, 1, 64),       # a single cached key
+    (1, 32, 1, 4, 3000, 128),  # 128 query rows per KV head (the tensor-core tile)
+    (1, 64, 2, 4, 2000, 64),   # 128 rows at d = 64
+    (1, 8, 1, 16, 1029, 128),  # one-tile splits: the last holds 5 keys, which 11 of the queries do not see
 ]
 
 
