@@ -25,7 +25,6 @@
 #include "bwd_sm100.cuh"
 #include "bwd2_sm100.cuh"
 #include "bwd256_sm100.cuh"
-#include "decode_sm100.cuh"
 #include "merge_sm100.cuh"
 
 namespace {
@@ -73,16 +72,6 @@ int check_device(int* dev_out) {
   return FA_OK;
 }
 
-// Dynamic shared memory of the KV-cache split kernels, one per row bucket.
-template <int HD, typename Set>
-void set_decode_attributes(Set& set) {
-  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 4>), fa::DecodeCfg<HD, 4>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 8>), fa::DecodeCfg<HD, 8>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 16>), fa::DecodeCfg<HD, 16>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 32>), fa::DecodeCfg<HD, 32>::SMEM_BYTES);
-  set(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, 64>), fa::DecodeCfg<HD, 64>::SMEM_BYTES);
-}
-
 // Opt every kernel into its dynamic shared memory, once per device.
 int prepare_kernels(int dev) {
   static std::mutex mu;
@@ -104,7 +93,7 @@ int prepare_kernels(int dev) {
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<64>), fa::fwd_f32_smem_bytes<64>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<128>), fa::fwd_f32_smem_bytes<128>());
   set(reinterpret_cast<const void*>(&fa::fa_fwd_f32_kernel<256>), fa::fwd_f32_smem_bytes<256>());
-  set_decode_attributes<256>(set);
+  set(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<256, true>), fa::FwdCfg<256, true>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64>), fa::Bwd2Cfg<64>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128>), fa::Bwd2Cfg<128>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64, true>), fa::Bwd2Cfg<64>::SMEM_BYTES);
@@ -684,25 +673,6 @@ int run_bwd_varlen(const void* q, const void* k, const void* v, const void* o, c
   return FA_OK;
 }
 
-// KV-cache forward: R query rows per KV head, S key splits of L keys (L a
-// multiple of 64). About four CTAs per SM of a 148-SM part, at least 256 keys
-// per split; a pure function of the sizes.
-struct DecodePlan {
-  int R, S, L;
-};
-
-DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk) {
-  DecodePlan dp;
-  dp.R = (Hq / Hkv) * Nq;
-  const long long pairs = static_cast<long long>(B) * Hkv;
-  const long long by_keys = std::max(1, (Nk + 255) / 256);
-  const long long by_sms = std::max(1LL, (592 + pairs - 1) / pairs);
-  const int s = static_cast<int>(std::min(by_keys, by_sms));
-  dp.L = ((Nk + s - 1) / s + 63) / 64 * 64;
-  dp.S = (Nk + dp.L - 1) / dp.L;
-  return dp;
-}
-
 // Validation of fa_fwd_kvcache's sizes: FA_OK, or the error to report.
 int check_kvcache_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype) {
   if (B < 0 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < Nq || d < 1) return FA_ERR_INVALID;
@@ -710,13 +680,12 @@ int check_kvcache_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, float sca
   if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_INVALID;
   if (static_cast<long long>(B) * Hq > INT32_MAX / 2 || Nk > INT32_MAX - 256) return FA_ERR_INVALID;
   if (dtype != FA_BF16 || (d != 64 && d != 128 && d != 256)) return FA_ERR_UNSUPPORTED;
-  // query rows per KV head: one 128-row MMA tile on the tensor cores (d = 64,
-  // 128), at most 64 rows in the d = 256 kernel
-  if (static_cast<long long>(Hq / Hkv) * Nq > (d == 256 ? 64 : 128)) return FA_ERR_UNSUPPORTED;
+  // query rows per KV head: one 128-row MMA tile
+  if (static_cast<long long>(Hq / Hkv) * Nq > 128) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
-// KV-cache forward on the tensor cores (d = 64, 128): one CTA per (batch,
+// KV-cache forward on the tensor cores: one CTA per (batch,
 // KV head, key split), one CTA per SM (its K/V ring fills shared memory and
 // it allocates all of TMEM). The split count minimises the estimated time,
 // waves x (tiles per split + a fixed cost of about two tiles per CTA); a
@@ -743,17 +712,11 @@ DecodeTcPlan decode_tc_plan(int B, int Hkv, int Nk) {
   return best;
 }
 
-bool decode_on_tensor_cores(int d) { return d == 64 || d == 128; }
-
 size_t kvcache_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
-  if (decode_on_tensor_cores(d)) {
-    // split parts of O (bf16) and LSE (f32) for the merge; none with one split
-    const DecodeTcPlan tp = decode_tc_plan(B, Hkv, Nk);
-    if (tp.S == 1) return 0;
-    return static_cast<size_t>(tp.S) * B * Hq * Nq * (2 * static_cast<size_t>(d) + 4);
-  }
-  const DecodePlan dp = decode_plan(B, Hq, Hkv, Nq, Nk);
-  return sizeof(float) * static_cast<size_t>(B) * Hkv * dp.S * dp.R * (static_cast<size_t>(d) + 2);
+  // split parts of O (bf16) and LSE (f32) for the merge; none with one split
+  const DecodeTcPlan tp = decode_tc_plan(B, Hkv, Nk);
+  if (tp.S == 1) return 0;
+  return static_cast<size_t>(tp.S) * B * Hq * Nq * (2 * static_cast<size_t>(d) + 4);
 }
 
 template <int HD>
@@ -799,63 +762,6 @@ int launch_decode_tc(const void* q, const void* k, const void* v, void* o, float
       cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return FA_ERR_CUDA;
   return launch_merge<HD>(o_part, lse_part, tp.S, rows_total, o, lse, num_sms, stream);
-}
-
-template <int HD, int RB>
-int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* ws, int B, int Hq,
-                  int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream) {
-  using C = fa::DecodeCfg<HD, RB>;
-  const DecodePlan dp = decode_plan(B, Hq, Hkv, Nq, Nk);
-  const uint64_t rows_kv = static_cast<uint64_t>(B) * Hkv;
-  CUtensorMap mk, mv;
-  int rc = make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Nk, rows_kv, 64, C::BK);
-  if (rc == FA_OK) rc = make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Nk, rows_kv, 64, C::BK);
-  if (rc != FA_OK) return rc;
-  float* part_o = static_cast<float*>(ws);
-  float* part_ml = part_o + rows_kv * dp.S * dp.R * HD;
-  fa::DecodeParams p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.part_o = part_o;
-  p.part_ml = part_ml;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.Nq = Nq;
-  p.Nk = Nk;
-  p.R = dp.R;
-  p.S = dp.S;
-  p.L = dp.L;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.causal = causal;
-  p.timeout_ns = timeout_now();
-  if (rows_kv > 65535) return FA_ERR_UNSUPPORTED;  // grid y
-  const dim3 grid(static_cast<unsigned>(dp.S), static_cast<unsigned>(rows_kv));
-  fa::fa_decode_split_kernel<HD, RB><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mk, mv, p);
-  if ((rc = launch_status(reinterpret_cast<const void*>(&fa::fa_decode_split_kernel<HD, RB>))) != FA_OK) return rc;
-  fa::DecodeMergeParams mp;
-  mp.part_o = part_o;
-  mp.part_ml = part_ml;
-  mp.o = static_cast<__nv_bfloat16*>(o);
-  mp.lse = lse;
-  mp.Hq = Hq;
-  mp.Hkv = Hkv;
-  mp.Nq = Nq;
-  mp.R = dp.R;
-  mp.S = dp.S;
-  mp.rows = static_cast<int>(rows_kv * dp.R);
-  fa::fa_decode_merge_kernel<HD><<<static_cast<unsigned>((mp.rows + 7) / 8), 256, 0, stream>>>(mp);
-  return launch_status();
-}
-
-// Row bucket of the split kernel: the smallest of 4, 8, 16, 32, 64 that holds R.
-template <int HD>
-int launch_decode_rows(const void* q, const void* k, const void* v, void* o, float* lse, void* ws, int B, int Hq,
-                       int Hkv, int Nq, int Nk, float scale, int causal, cudaStream_t stream) {
-  const int R = (Hq / Hkv) * Nq;
-  if (R <= 4) return launch_decode<HD, 4>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
-  if (R <= 8) return launch_decode<HD, 8>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
-  if (R <= 16) return launch_decode<HD, 16>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
-  if (R <= 32) return launch_decode<HD, 32>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
-  return launch_decode<HD, 64>(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, scale, causal, stream);
 }
 
 // Checks shared by the backward entry points. `ptrs` must all be 16-byte aligned and non-null.
@@ -1204,7 +1110,7 @@ int fa_fwd_kvcache(const void* q, const void* k, const void* v, void* o, float* 
   switch (d) {
     case 64: return launch_decode_tc<64>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
     case 128: return launch_decode_tc<128>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
-    default: return launch_decode_rows<256>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
+    default: return launch_decode_tc<256>(q, k, v, o, lse, workspace, B, Hq, Hkv, Nq, Nk, scale, causal, s);
   }
 }
 

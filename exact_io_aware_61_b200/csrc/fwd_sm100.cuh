@@ -39,7 +39,7 @@ template <int HD, bool DECODE = false>
 struct FwdCfg {
   static constexpr int BM = 128;  // query rows per CTA
   static constexpr int BN = 128;  // keys per tile
-  static constexpr int STAGES = DECODE ? (HD == 64 ? 6 : 3) : (HD == 64 ? 4 : (HD == 128 ? 2 : 1));
+  static constexpr int STAGES = DECODE ? (HD == 64 ? 6 : (HD == 128 ? 3 : 1)) : (HD == 64 ? 4 : (HD == 128 ? 2 : 1));
   static constexpr int Q_BYTES = BM * HD * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
   static constexpr int SMEM_BYTES = 1024 + Q_BYTES + 2 * STAGES * KV_BYTES;

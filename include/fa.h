@@ -335,18 +335,12 @@ FA_API int fa_bwd_varlen(const void* q, const void* k, const void* v, const void
 
 /*
  * fa_fwd_kvcache_workspace_size -- bytes of device workspace fa_fwd_kvcache
- * needs, a pure function of the sizes (0 for invalid sizes):
- *   d = 64, 128: per key split, the split's normalised output rows (bf16)
- *     and LSE (float32) of all B * Hq * Nq query rows:
- *     S * B * Hq * Nq * (2 d + 4) bytes, and 0 when S = 1. The keys are cut
- *     into S splits of T tiles of 128 keys; (S, T) minimise
- *     ceil(B * Hkv * S / 148) * (T + 2) over S = 1 .. min(tiles, 128),
- *     T = ceil(tiles / S), S then reduced to ceil(tiles / T);
- *   d = 256: per key split, the softmax state (max, sum, unnormalised output
- *     row) of each of the R = (Hq / Hkv) * Nq query rows of a KV head,
- *     float32: B * Hkv * S * R * (d + 2) * 4 bytes, with
- *     S = min(ceil(Nk / 256), ceil(592 / (B * Hkv))), at least 1, then the
- *     keys cut into S chunks of a multiple of 64.
+ * needs, a pure function of the sizes (0 for invalid sizes): per key split,
+ * the split's normalised output rows (bf16) and LSE (float32) of all
+ * B * Hq * Nq query rows, S * B * Hq * Nq * (2 d + 4) bytes, and 0 when
+ * S = 1. The keys are cut into S splits of T tiles of 128 keys; (S, T)
+ * minimise ceil(B * Hkv * S / 148) * (T + 2) over S = 1 .. min(tiles, 128),
+ * T = ceil(tiles / S), S then reduced to ceil(tiles / T).
  */
 FA_API size_t fa_fwd_kvcache_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
 
@@ -370,12 +364,10 @@ FA_API size_t fa_fwd_kvcache_workspace_size(int B, int Hq, int Hkv, int Nq, int 
  * ("A pinch of math: making the softmax work in pieces"). Two kernels run in
  * stream order: one CTA per (batch, KV head, key split) computes each split's
  * result for all R = (Hq / Hkv) * Nq query rows of the KV head (K and V are
- * read from HBM once), then a merge kernel writes O and LSE (with one split,
- * d <= 128, the first kernel writes them itself). At d = 64 and 128 the first
- * kernel runs on the tensor cores with the R rows as one 128-row tile; at
- * d = 256 on the CUDA cores. Supports dtype FA_BF16 with d in {64, 128, 256},
- * R <= 128 (d = 64, 128) or R <= 64 (d = 256); other cases return
- * FA_ERR_UNSUPPORTED. Nq > Nk or Nq < 1 returns FA_ERR_INVALID; B == 0 is a
+ * read from HBM once), then a merge kernel writes O and LSE (with one split
+ * the first kernel writes them itself). The first kernel runs on the tensor
+ * cores with the R rows as one 128-row tile. Supports dtype FA_BF16 with d in
+ * {64, 128, 256} and R <= 128; other cases return FA_ERR_UNSUPPORTED. Nq > Nk or Nq < 1 returns FA_ERR_INVALID; B == 0 is a
  * no-op. The workspace may be null when its size is 0. On error nothing is
  * written.
  */

@@ -407,6 +407,7 @@ KVCACHE_SHAPES = [  # (B, Hq, Hkv, Nq, Nk, d)
     (1, 32, 1, 4, 3000, 128),  # 128 query rows per KV head (the tensor-core tile)
     (1, 64, 2, 4, 2000, 64),   # 128 rows at d = 64
     (1, 8, 1, 16, 1029, 128),  # one-tile splits: the last holds 5 keys, which 11 of the queries do not see
+    (1, 32, 2, 8, 3000, 256),  # 128 rows at d = 256
 ]
 
 
