@@ -403,21 +403,6 @@ FA_DEV float ex2_approx(float x) {  // 2^x on the SFU; ex2(-inf) = +0
   return y;
 }
 
-// 2^x on the FMA pipe, for x in [-126, 8]: x = j + f with j = round(x) and
-// f in [-0.5, 0.5]; 2^f by a cubic whose coefficients were fitted here by a
-// Remez exchange for minimax relative error on [-0.5, 0.5] (7.5e-5, far
-// below the bf16 rounding the results go through); 2^j is added to the
-// exponent field. Used for part of a tile's exponentials so that the SFU,
-// which the rest go to, is not the only unit doing them. Smaller x is
-// clamped to -126 (2^-126, negligible next to the values it is summed with).
-FA_DEV float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;  // 1.5 * 2^23: the sum's low bits hold round(x)
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.05517166906f, f, 0.2426111222f), f, 0.6932609855f), f, 0.9999280735f);
-  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
-}
-
 // Two floats -> packed bf16x2 (round to nearest even); `lo` in bits 0..15.
 FA_DEV uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
