@@ -44,6 +44,11 @@ struct Fwd2Cfg {
   static_assert(128 * (2 * SOFTMAX_REGS + OTHER_REGS) <= THREADS * LAUNCH_REGS, "register split exceeds launch");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TMEM_O = 256;  // O0 at 256, O1 at 256 + HD
+  // d = 64 leaves room for P in its own columns (P0 at 384, P1 at 448), so
+  // S(j+1) can be computed as soon as the softmax has read S(j) instead of
+  // after P(j)V(j); at d = 128 P overwrites S.
+  static constexpr bool SEP_P = HD == 64;
+  static constexpr uint32_t TMEM_P = 384;
   static constexpr float RESCALE_THRESHOLD = 8.0f;
   static constexpr int HEAD_GROUP = 8;  // heads scheduled together (K/V stay in L2)
 };
@@ -128,7 +133,7 @@ __global__ void __launch_bounds__(384, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q, bar_kfull[KST], bar_kempty[KST], bar_vfull[VST], bar_vempty[VST];
-  __shared__ uint64_t bar_sfull[2], bar_pfull[2], bar_odone[2], bar_drain;
+  __shared__ uint64_t bar_sfull[2], bar_pfull[2], bar_odone[2], bar_sfree[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -228,6 +233,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(smem_u32(&bar_sfull[t]), 1);
       mbar_init(smem_u32(&bar_pfull[t]), 128);
       mbar_init(smem_u32(&bar_odone[t]), 1);
+      mbar_init(smem_u32(&bar_sfree[t]), 128);
     }
     mbar_init(smem_u32(&bar_drain), 1);
     fence_mbar_init();
@@ -314,6 +320,22 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; ok && j < n_max; ++j) {
         const int s = j % VST;
         bool v_ready = false, k_next_ready = false;
+        if constexpr (C::SEP_P) {
+          // S(j+1) of each tile as soon as its softmax has read S(j); P(j)
+          // has its own columns, so it does not wait for P(j)V(j)
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j + 1 >= n_t[t]) continue;
+            if (!mbar_wait(smem_u32(&bar_sfree[t]), j & 1, wc)) { ok = false; break; }
+            if (!k_next_ready) {
+              if (!mbar_wait(smem_u32(&bar_kfull[(j + 1) % KST]), ((j + 1) / KST) & 1, wc)) { ok = false; break; }
+              k_next_ready = true;
+            }
+            tc_fence_after();
+            issue_s(t, j + 1);
+          }
+          if (!ok) break;
+          if (k_next_ready) mma_commit(smem_u32(&bar_kempty[(j + 1) % KST]));
+        }
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= n_t[t]) continue;
           if (!mbar_wait(smem_u32(&bar_pfull[t]), j & 1, wc)) { ok = false; break; }
@@ -323,12 +345,13 @@ __global__ void __launch_bounds__(384, 1)
           }
           tc_fence_after();
           const uint32_t vb = sV + s * C::KV_BYTES;
+          const uint32_t pa = tmem + (C::SEP_P ? C::TMEM_P + t * 64 : t * 128);
 #pragma unroll
           for (int kk = 0; kk < C::BN / 16; ++kk)
-            mma_bf16_ts(tmem + C::TMEM_O + t * HD, tmem + t * 128 + kk * 8,
-                        sdesc_sw128(vb + kk * 2048, C::BN * 128, 1024), idesc_pv, (j > 0 || kk > 0));
+            mma_bf16_ts(tmem + C::TMEM_O + t * HD, pa + kk * 8, sdesc_sw128(vb + kk * 2048, C::BN * 128, 1024),
+                        idesc_pv, (j > 0 || kk > 0));
           mma_commit(smem_u32(&bar_odone[t]));
-          if (j + 1 < n_t[t]) {
+          if (!C::SEP_P && j + 1 < n_t[t]) {
             if (!k_next_ready) {
               if (!mbar_wait(smem_u32(&bar_kfull[(j + 1) % KST]), ((j + 1) / KST) & 1, wc)) { ok = false; break; }
               k_next_ready = true;
@@ -339,7 +362,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         mma_commit(smem_u32(&bar_vempty[s]));
-        if (k_next_ready) mma_commit(smem_u32(&bar_kempty[(j + 1) % KST]));
+        if (!C::SEP_P && k_next_ready) mma_commit(smem_u32(&bar_kempty[(j + 1) % KST]));
       }
       // no MMA may be in flight when tensor memory is released
       mma_commit(smem_u32(&bar_drain));
@@ -363,6 +386,10 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld128(s_addr, sr);
+      if constexpr (C::SEP_P) {  // S(j) is in registers: its columns may take S(j+1)
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bar_sfree[t]));
+      }
       const int key0 = j * C::BN;
       if ((p.causal && key0 + C::BN > kv_off + q0 + t * C::BM) || key0 + C::BN > k_len) {
         const int lim = min(p.causal ? kv_off + row + 1 : k_len, k_len) - key0;
@@ -411,6 +438,13 @@ __global__ void __launch_bounds__(384, 1)
       float s0, s1;
       unpack2(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), s0, s1);
       l = l * alpha + (s0 + s1);
+      if constexpr (C::SEP_P) {
+        // P(j) goes to its own columns, which P(j-1)V(j-1) reads: wait for it
+        if (j > 0) {
+          if (!warp_wait(smem_u32(&bar_odone[t]), (j - 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+        }
+      }
       {
         uint32_t h0[32], h1[32];
 #pragma unroll
@@ -418,12 +452,14 @@ __global__ void __launch_bounds__(384, 1)
           h0[i] = pk[i];
           h1[i] = pk[32 + i];
         }
-        tmem_st32(s_addr, h0);
-        tmem_st32(s_addr + 32, h1);
+        const uint32_t p_addr = C::SEP_P ? tmem + lane_base + C::TMEM_P + t * 64 : s_addr;
+        tmem_st32(p_addr, h0);
+        tmem_st32(p_addr + 32, h1);
       }
       if (rescale) {
-        // o was last written by P_{j-1} V_{j-1}: wait for it, then scale by alpha
-        if (!warp_wait(smem_u32(&bar_odone[t]), (j - 1) & 1, wc)) { ok = false; break; }
+        // o was last written by P_{j-1} V_{j-1}: wait for it (done above when
+        // P has its own columns), then scale by alpha
+        if (!C::SEP_P && !warp_wait(smem_u32(&bar_odone[t]), (j - 1) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         const uint64_t a2 = pack2(alpha, alpha);
 #pragma unroll

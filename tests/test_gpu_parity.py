@@ -276,6 +276,33 @@ def test_bwd_causal_b1_h8_kv2_n4096_d256_all_heads(fa):
         assert _rel_fro(got_v[:, hk:hk + 1], rv) <= GRAD_TOL
 
 
+def test_bwd_causal_b1_h16_kv4_n8192_d256_one_group_full(fa):
+    """The d = 256 GQA configuration at 8k tokens: dK and dV of one KV head
+    (the last, so its CTAs run after every other group's) and the dQ of its
+    four query heads against the oracle in full; sampled dQ rows on every
+    other head."""
+    B, Hq, Hkv, N, d = 1, 16, 4, 8192, 256
+    inp = INP.make_inputs(B, Hq, Hkv, N, d, "bf16", seed=8192 + d, grad=True)
+    dq, dk, dv = _run_bwd(fa, inp, True, d ** -0.5)
+    g = Hq // Hkv
+    hk = Hkv - 1
+    hs = slice(hk * g, (hk + 1) * g)
+    q, k, v, do = (INP.as_f64(inp[n][:, sl]) for n, sl in (("q", hs), ("k", slice(hk, hk + 1)),
+                                                            ("v", slice(hk, hk + 1)), ("do", hs)))
+    rq, rk, rv, _ = ORACLE.attention_backward(q, k, v, do, d ** -0.5, True)
+    assert _rel_fro(INP.as_f64(dq[:, hs]), rq) <= GRAD_TOL
+    assert _rel_fro(INP.as_f64(dk[:, hk:hk + 1]), rk) <= GRAD_TOL
+    assert _rel_fro(INP.as_f64(dv[:, hk:hk + 1]), rv) <= GRAD_TOL
+    rng = np.random.default_rng(11)
+    for h in range(0, hk * g):
+        rows = sorted(set([0, 63, 64, N - 1] + [int(x) for x in rng.integers(0, N, 6)]))
+        hkv = h // g
+        qh, kh, vh, doh = (INP.as_f64(inp[n][:, sl]) for n, sl in (("q", slice(h, h + 1)), ("k", slice(hkv, hkv + 1)),
+                                                                   ("v", slice(hkv, hkv + 1)), ("do", slice(h, h + 1))))
+        rqr, _, _ = ORACLE.attention_backward_rows(qh, kh, vh, doh, d ** -0.5, True, 0, 0, rows)
+        assert _rel_fro(INP.as_f64(dq[0, h, rows]), rqr) <= GRAD_TOL, h
+
+
 def test_bwd_causal_b2_h32_n8192_d128(fa):
     """The benchmark backward (B=2, H=32, N=8192, d=128, causal), the shape
     bench.py times. Full fp64 dQ, dK, dV on one head from every group of 8
