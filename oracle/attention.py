@@ -95,6 +95,7 @@ __all__ = [
     "merge_partial_states",
     "attention_forward_positions",
     "merge_outputs",
+    "attention_backward_block",
 ]
 
 
@@ -494,4 +495,37 @@ def attention_backward_varlen(q, k, v, do, cu_q, cu_k, scale: float, causal: boo
             ds = score_gradient(p, dp, D)
             dq[q0:q1, h] = scale * (ds @ ks)
             dk[k0:k1, hk] += scale * (ds.T @ qs)
+    return dq, dk, dv
+
+
+def attention_backward_block(q, k, v, do, lse, D, q_pos, k_pos, scale: float, causal: bool):
+    """The share of one key block in the gradients, given the full rows' statistics.
+
+    ``q``, ``do`` are ``[B, Hq, Nq, d]`` at positions ``q_pos``; ``k``, ``v``
+    are ``[B, Hkv, Nk, d]`` at positions ``k_pos`` (one block of a longer key
+    sequence); ``lse`` and ``D = rowsum(dO * O)`` are ``[B, Hq, Nq]`` for the
+    queries' whole rows (every key block). With those, the weights of the
+    block's keys are ``P = exp(scale S - LSE)`` (masked entries 0), and the
+    block adds ``dQ += scale dS K``, ``dK = scale dS^T Q``, ``dV = P^T dO``
+    with ``dS = P * (dP - D)``, ``dP = dO V^T`` (the formulas of
+    :func:`attention_backward`, restricted to the block's keys). Summed over
+    a partition of the keys they give :func:`attention_backward`. Returns
+    ``(dQ [B,Hq,Nq,d], dK [B,Hkv,Nk,d], dV [B,Hkv,Nk,d])``.
+    """
+    q, k, v, do, lse, D = (_f64(x) for x in (q, k, v, do, lse, D))
+    B, Hq = q.shape[:2]
+    Hkv = k.shape[1]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = kv_head_of(h, Hq, Hkv)
+            s = masked_scores(q[b, h], k[b, hk], scale, causal, rows=q_pos, keys=k_pos)
+            with np.errstate(invalid="ignore"):
+                p = np.where(np.isfinite(s), np.exp(s - lse[b, h][:, None]), 0.0)
+            dv[b, hk] += p.T @ do[b, h]
+            ds = score_gradient(p, do[b, h] @ v[b, hk].T, D[b, h])
+            dq[b, h] = scale * (ds @ k[b, hk])
+            dk[b, hk] += scale * (ds.T @ q[b, h])
     return dq, dk, dv

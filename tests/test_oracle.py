@@ -461,7 +461,35 @@ def check_varlen_backward_finite_differences(o):
             assert np.max(np.abs(num - grad)) < 1e-7, name
 
 
+
+def check_backward_blocks_sum_to_the_full_backward(o):
+    # Striped key blocks (W = 3) of every query shard, each with the full rows'
+    # LSE and D, add up to the (pinned) backward of the unsharded problem.
+    q, k, v = _qkv(B=1, Hq=4, Hkv=2, N=12, d=5, seed=113)
+    do = _rand((1, 4, 12, 5), 114)
+    W = 3
+    for causal in (False, True):
+        fo, fl = o.attention_forward(q, k, v, 0.45, causal)
+        rq, rk, rv, D = o.attention_backward(q, k, v, do, 0.45, causal)
+        dq = np.zeros_like(q)
+        dk = np.zeros_like(k)
+        dv = np.zeros_like(v)
+        for r in range(W):
+            qp = r + W * np.arange(12 // W)
+            for c in range(W):
+                kp = c + W * np.arange(12 // W)
+                bq, bk, bv = o.attention_backward_block(q[:, :, r::W], k[:, :, c::W], v[:, :, c::W], do[:, :, r::W],
+                                                        fl[:, :, r::W], D[:, :, r::W], qp, kp, 0.45, causal)
+                dq[:, :, r::W] += bq
+                dk[:, :, c::W] += bk
+                dv[:, :, c::W] += bv
+        assert np.max(np.abs(dq - rq)) < 1e-12
+        assert np.max(np.abs(dk - rk)) < 1e-12
+        assert np.max(np.abs(dv - rv)) < 1e-12
+
+
 ALL_CHECKS = [
+    check_backward_blocks_sum_to_the_full_backward,
     check_varlen_backward_square_sequences_are_the_square_backward,
     check_varlen_backward_finite_differences,
     check_positions_reduce_to_square_and_kvcache,
@@ -544,6 +572,12 @@ def _mut_varlen_backward_top_left(q, k, v, do, cu_q, cu_k, scale, causal):  # qu
     return dq, dk, dv
 
 
+def _mut_block_backward_local_lse(q, k, v, do, lse, D, q_pos, k_pos, scale, causal):  # block's own LSE
+    _, local = ORACLE.attention_forward_positions(q, k, v, q_pos, k_pos, scale, causal)
+    return ORIG["attention_backward_block"](q, k, v, do, np.where(np.isfinite(local), local, 0.0), D, q_pos, k_pos,
+                                            scale, causal)
+
+
 def _mut_positions_ignore_keys(q, k, v, q_pos, k_pos, scale, causal):  # key positions taken as 0..Nk-1
     return ORIG["attention_forward_positions"](q, k, v, q_pos, np.arange(np.shape(k)[2]), scale, causal)
 
@@ -598,7 +632,7 @@ def _mut_merge_no_rescale(ms, ls, os):  # sums added without the exp(m_s - M) fa
 
 
 ORIG = {name: getattr(ORACLE, name) for name in ("masked_scores", "softmax_rows", "score_gradient", "kv_head_of",
-                                                 "attention_forward_positions")}
+                                                 "attention_forward_positions", "attention_backward_block")}
 
 MUTATIONS = [
     ("score_gradient", _mut_drop_D),
@@ -615,6 +649,7 @@ MUTATIONS = [
     ("attention_forward_positions", _mut_positions_ignore_keys),
     ("merge_outputs", _mut_merge_outputs_plain_mean),
     ("attention_backward_varlen", _mut_varlen_backward_top_left),
+    ("attention_backward_block", _mut_block_backward_local_lse),
 ]
 
 
