@@ -24,11 +24,13 @@ from ._lib import (  # noqa: F401
     fa_bwd_main,
     fa_bwd_dq,
     fa_bwd_noalloc,
+    fa_bwd_partial,
     fa_bwd_prep,
     fa_bwd_varlen,
     fa_bwd_varlen_workspace_size,
     fa_bwd_workspace_size,
     fa_fwd,
+    fa_f32_to_bf16,
     fa_fwd_kvcache,
     fa_fwd_partial,
     fa_fwd_varlen,

@@ -33,6 +33,8 @@ EXPORTED = (
     "fa_bwd_workspace_size",
     "fa_bwd_varlen",
     "fa_bwd_varlen_workspace_size",
+    "fa_bwd_partial",
+    "fa_f32_to_bf16",
     "fa_fwd_kvcache",
     "fa_fwd_kvcache_workspace_size",
     "fa_status_string",
@@ -84,6 +86,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i,
                                       vp, sz, i, vp]
         lib.fa_bwd_varlen.restype = i
+        lib.fa_bwd_partial.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, i, vp]
+        lib.fa_bwd_partial.restype = i
+        lib.fa_f32_to_bf16.argtypes = [vp, vp, sz, vp]
+        lib.fa_f32_to_bf16.restype = i
         lib.fa_bwd_varlen_workspace_size.argtypes = [i, i, i, i, i, i]
         lib.fa_bwd_varlen_workspace_size.restype = sz
         lib.fa_bwd_workspace_size.argtypes = [i, i, i, i, i]
@@ -263,6 +269,34 @@ def backward_bnhd(q, k, v, o, lse, do, causal: bool = False, scale: float | None
                                  o.reshape(B * N, Hq, d), lse.reshape(B * N, Hq), do.reshape(B * N, Hq, d), offs, offs,
                                  N, N, causal, scale, stream)
     return dq.view(B, N, Hq, d), dk.view(B, N, Hkv, d), dv.view(B, N, Hkv, d)
+
+
+def fa_bwd_partial(q, k, v, do, dk_acc, dv_acc, workspace, causal: bool, scale: float, diag_offset: int,
+                   stream=None) -> None:
+    """Call ``fa_bwd_partial``: add one key block's dK, dV into the f32 ``dk_acc``, ``dv_acc`` and its dQ into
+    the workspace accumulator (after ``fa_bwd_prep``)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("do", do), ("dk_acc", dk_acc), ("dv_acc", dv_acc)):
+        _check_tensor(name, t, q.device)
+    if dk_acc.dtype != torch.float32 or dv_acc.dtype != torch.float32:
+        raise TypeError("dk_acc and dv_acc must be float32")
+    B, Hq, N, d = q.shape
+    ws_ptr, ws_bytes = _ws(workspace)
+    rc = load().fa_bwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk_acc), _ptr(dv_acc), ws_ptr, ws_bytes, B,
+                               Hq, k.shape[1], N, d, float(scale), int(bool(causal)), int(diag_offset),
+                               _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_partial")
+
+
+def fa_f32_to_bf16(src, dst, stream=None) -> None:
+    """Call ``fa_f32_to_bf16``: dst (bf16) = src (f32), same number of elements."""
+    for name, t in (("src", src), ("dst", dst)):
+        _check_tensor(name, t, src.device)
+    if src.dtype != torch.float32 or dst.dtype != torch.bfloat16 or src.numel() != dst.numel():
+        raise TypeError("src must be float32 and dst bfloat16 with as many elements")
+    rc = load().fa_f32_to_bf16(_ptr(src), _ptr(dst), src.numel(), ctypes.c_void_p(_stream_ptr(stream)))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_f32_to_bf16")
 
 
 def fa_bwd_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:

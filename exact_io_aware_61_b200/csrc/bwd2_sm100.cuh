@@ -101,6 +101,10 @@ struct Bwd2Params {
   const int* cu_q;
   const int* cu_k;
   int batch, total_q, total_k, max_seqlen_q, max_seqlen_k;
+  // PARTIAL kernel (one key block of a longer sequence): the causal diagonal
+  // moved by diag_shift keys, query i sees key j iff j <= i + diag_shift; dK
+  // and dV are added into dk_acc, dv_acc (f32, not zeroed here).
+  int diag_shift;
 };
 
 
@@ -108,7 +112,8 @@ struct Bwd2Params {
 // VARLEN: packed variable-length batches (see Bwd2Params); the tensor maps are
 // then rank-3 views {d, heads, tokens} with a {64 or 32, 1, 128} box, which
 // lands in shared memory like the dense box.
-template <int HD, bool VARLEN = false>
+// PARTIAL: dense layout, shifted diagonal, dK/dV added into f32 accumulators.
+template <int HD, bool VARLEN = false, bool PARTIAL = false>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd2_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -184,24 +189,24 @@ __global__ void __launch_bounds__(512, 1)
   const int h_first = slice * heads;
   // query i of the sequence sits at key position kv_off + i (its last
   // positions when it has fewer queries than keys)
-  const int kv_off = k_len - q_len;
+  const int kv_off = k_len - q_len + (PARTIAL ? p.diag_shift : 0);
   const int i_begin = p.causal ? max(0, (k0 - kv_off) / 128) : 0;  // first query tile that sees key tile kt
   const int per_head = (q_len + 127) / 128 - i_begin;
   const int steps = heads * max(per_head, 0);
-  if constexpr (VARLEN) {
-    if (steps == 0) {
-      // a sequence without queries: its keys get zero gradients (already
-      // zero in the f32 accumulators when the group is split)
-      if (p.head_split == 1 && threadIdx.x < 256) {
-        const int key = k0 + (threadIdx.x & 127);
-        if (key < k_len) {
-          __nv_bfloat16* out = (threadIdx.x < 128 ? p.dv : p.dk) + (static_cast<size_t>(k_tok + key) * p.Hkv + hkv) * HD;
+  if (steps == 0) {
+    // no query sees this key tile (a sequence without queries, or a shifted
+    // diagonal): its keys get zero gradients, already zero (or left as they
+    // are) in f32 accumulators
+    if (p.head_split == 1 && !PARTIAL && threadIdx.x < 256) {
+      const int key = k0 + (threadIdx.x & 127);
+      if (key < k_len) {
+        const size_t row = VARLEN ? static_cast<size_t>(k_tok + key) * p.Hkv + hkv : static_cast<size_t>(bhkv) * p.N + key;
+        __nv_bfloat16* out = (threadIdx.x < 128 ? p.dv : p.dk) + row * HD;
 #pragma unroll
-          for (int i = 0; i < HD / 8; ++i) reinterpret_cast<uint4*>(out)[i] = make_uint4(0u, 0u, 0u, 0u);
-        }
+        for (int i = 0; i < HD / 8; ++i) reinterpret_cast<uint4*>(out)[i] = make_uint4(0u, 0u, 0u, 0u);
       }
-      return;
     }
+    return;
   }
 
   WaitCtl wc{&abort_flag, p.timeout_ns};
@@ -400,7 +405,9 @@ __global__ void __launch_bounds__(512, 1)
       // or, variable-length, a query past the sequence's end (its workspace
       // row may belong to the next sequence, so the weight is zeroed here;
       // dense padding rows have LSE = +inf and weigh 0 already)
-      const bool mask = VARLEN ? (p.causal && k0 + 127 > kv_off + q0) || q0 + 128 > q_len : p.causal && q0 == k0;
+      const bool mask = VARLEN    ? (p.causal && k0 + 127 > kv_off + q0) || q0 + 128 > q_len
+                        : PARTIAL ? p.causal && k0 + 127 > kv_off + q0
+                                  : p.causal && q0 == k0;
       uint32_t pk[32];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
@@ -419,7 +426,8 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int qi = q0 + qa + e;
-              if (VARLEN ? (p.causal && key > kv_off + qi) || qi >= q_len : qi < key) pv[e] = 0.f;
+              if (VARLEN ? (p.causal && key > kv_off + qi) || qi >= q_len : PARTIAL ? key > kv_off + qi : qi < key)
+                pv[e] = 0.f;
             }
           }
           pk[u * 16 + 2 * x] = key_live ? pack_bf16x2(pv[0], pv[1]) : 0u;
@@ -472,13 +480,14 @@ __global__ void __launch_bounds__(512, 1)
       const size_t row_off = VARLEN ? (static_cast<size_t>(k_tok + (key_live ? key : 0)) * p.Hkv + hkv) * HD
                                     : (static_cast<size_t>(bhkv) * p.N + (key_live ? key : 0)) * HD;
       __nv_bfloat16* out = (half == 0 ? p.dv : p.dk) + row_off;
-      float* acc = p.head_split > 1 ? (half == 0 ? p.dv_acc : p.dk_acc) + row_off : nullptr;
+      const bool to_acc = p.head_split > 1 || PARTIAL;
+      float* acc = to_acc ? (half == 0 ? p.dv_acc : p.dk_acc) + row_off : nullptr;
       const uint32_t col = half == 0 ? C::T_DV : C::T_DK;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_base + col + c * 32, r);
-        if (p.head_split > 1) {
+        if (to_acc) {
           if (key_live) {
 #pragma unroll
             for (int x = 0; x < 8; ++x)

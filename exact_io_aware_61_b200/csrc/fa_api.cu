@@ -98,6 +98,8 @@ int prepare_kernels(int dev) {
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128>), fa::Bwd2Cfg<128>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64, true>), fa::Bwd2Cfg<64>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128, true>), fa::Bwd2Cfg<128>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<64, false, true>), fa::Bwd2Cfg<64>::SMEM_BYTES);
+  set(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<128, false, true>), fa::Bwd2Cfg<128>::SMEM_BYTES);
   set(reinterpret_cast<const void*>(&fa::fa_bwd256_main_kernel), fa::Bwd256Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return FA_ERR_CUDA;
   done[dev] = true;
@@ -411,15 +413,18 @@ struct BwdPlan {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  bool partial;  // the main stage is fa_bwd_partial's (shifted diagonal, dK/dV added into caller f32)
 };
 
 // stages: bit 0 prep, bit 1 main, bit 2 dQ conversion. Pointers a stage does not use may be null.
 template <int HD>
 int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const void* v, const void* o,
              const float* lse, const void* dO, void* dq, void* dk, void* dv, void* ws, int B, int Hq, int Hkv,
-             int N, float scale, int causal, cudaStream_t stream) {
+             int N, float scale, int causal, cudaStream_t stream, int diag_shift = 0, float* dk_acc = nullptr,
+             float* dv_acc = nullptr) {
   using C = fa::Bwd2Cfg<HD == 256 ? 128 : HD>;
   pl->stream = stream;
+  pl->partial = dk_acc != nullptr;
   pl->w = carve(ws, B, Hq, Hkv, N, HD);
   pl->kv_elems = static_cast<size_t>(B) * Hkv * static_cast<size_t>(N) * HD;
   pl->q_elems = static_cast<size_t>(B) * Hq * static_cast<size_t>(N) * HD;
@@ -483,9 +488,10 @@ int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const v
     // the assumption of exactly LAUNCH_REGS per thread at launch; a build
     // with another count would wait for ever, so it is refused here.
     cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD == 256 ? 128 : HD>)) !=
-        cudaSuccess)
-      return FA_ERR_CUDA;
+    const void* kernel = pl->partial
+                             ? reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD == 256 ? 128 : HD, false, true>)
+                             : reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD == 256 ? 128 : HD>);
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
     if (attr.numRegs != C::LAUNCH_REGS) {
       if (verbose()) std::fprintf(stderr, "fa: backward built with %d registers, expected %d\n", attr.numRegs,
                                   C::LAUNCH_REGS);
@@ -517,6 +523,11 @@ int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const v
     mp.scale = scale;
     mp.causal = causal;
     mp.timeout_ns = timeout_now();
+    mp.diag_shift = diag_shift;
+    if (pl->partial) {
+      mp.dk_acc = dk_acc;
+      mp.dv_acc = dv_acc;
+    }
     const long long blocks = static_cast<long long>(mp.num_tiles) * B * Hkv * pl->split;
     if (blocks > INT32_MAX) return FA_ERR_INVALID;
     pl->main_blocks = static_cast<unsigned>(blocks);
@@ -532,7 +543,7 @@ int launch_bwd_stages(const BwdPlan& pl, unsigned stages) {
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
   if (stages & 2u) {
-    if (pl.split > 1) {  // zero the f32 dK and dV accumulators (contiguous)
+    if (pl.split > 1 && !pl.partial) {  // zero the f32 dK and dV accumulators (contiguous)
       fa::fa_zero_f32_kernel<<<grid_stride_blocks(pl.kv_elems / 2), 256, 0, pl.stream>>>(pl.w.dk_acc,
                                                                                         pl.kv_elems / 2);
       if (launch_status() != FA_OK) return FA_ERR_CUDA;
@@ -541,6 +552,12 @@ int launch_bwd_stages(const BwdPlan& pl, unsigned stages) {
       fa::fa_bwd256_main_kernel<<<pl.main_blocks, fa::Bwd256Cfg::THREADS, fa::Bwd256Cfg::SMEM_BYTES, pl.stream>>>(
           pl.mq, pl.mk, pl.mv, pl.mdo, pl.mp256);
       if (launch_status(reinterpret_cast<const void*>(&fa::fa_bwd256_main_kernel)) != FA_OK) return FA_ERR_CUDA;
+    } else if (pl.partial) {
+      fa::fa_bwd2_main_kernel<HD, false, true><<<pl.main_blocks, C::THREADS, C::SMEM_BYTES, pl.stream>>>(
+          pl.mq, pl.mk, pl.mv, pl.mdo, pl.mdq, pl.mp);
+      if (launch_status(reinterpret_cast<const void*>(&fa::fa_bwd2_main_kernel<HD, false, true>)) != FA_OK)
+        return FA_ERR_CUDA;
+      return FA_OK;  // dK, dV stay in the caller's f32 accumulators
     } else {
       fa::fa_bwd2_main_kernel<HD><<<pl.main_blocks, C::THREADS, C::SMEM_BYTES, pl.stream>>>(pl.mq, pl.mk, pl.mv,
                                                                                             pl.mdo, pl.mdq, pl.mp);
@@ -903,6 +920,41 @@ int fa_merge_partials(const void* o_parts, const float* lse_parts, int n_parts, 
     case 128: return launch_merge<128>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
     default: return launch_merge<256>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
   }
+}
+
+int fa_bwd_partial(const void* q, const void* k, const void* v, const void* dO, float* dk_acc, float* dv_acc,
+                   void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
+                   int causal, int diag_offset, int dtype, fa_stream_t stream) {
+  int dev = 0;
+  int rc = check_bwd({q, k, v, dO, dk_acc, dv_acc}, workspace, workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype,
+                     &dev);
+  if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // offsets beyond +-N change nothing; clamping keeps the kernel's index sums in range
+  const int shift = causal ? std::max(-N, std::min(N, diag_offset)) : 0;
+  BwdPlan pl;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) {
+    if ((rc = plan_bwd<64>(&pl, 2u, q, k, v, nullptr, nullptr, dO, nullptr, nullptr, nullptr, workspace, B, Hq, Hkv, N,
+                           scale, causal, s, shift, dk_acc, dv_acc)) != FA_OK)
+      return rc;
+    return launch_bwd_stages<64>(pl, 2u);
+  }
+  if ((rc = plan_bwd<128>(&pl, 2u, q, k, v, nullptr, nullptr, dO, nullptr, nullptr, nullptr, workspace, B, Hq, Hkv, N,
+                          scale, causal, s, shift, dk_acc, dv_acc)) != FA_OK)
+    return rc;
+  return launch_bwd_stages<128>(pl, 2u);
+}
+
+int fa_f32_to_bf16(const float* src, void* dst, size_t n, fa_stream_t stream) {
+  if (n == 0) return FA_OK;
+  if (n % 4 != 0 || !aligned16(src) || !aligned16(dst)) return FA_ERR_INVALID;
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  fa::fa_bwd_dq_kernel<<<grid_stride_blocks(n / 4), 256, 0, s>>>(src, static_cast<__nv_bfloat16*>(dst), n / 4);
+  return launch_status();
 }
 
 size_t fa_bwd_varlen_workspace_size(int batch, int total_q, int total_k, int Hq, int Hkv, int d) {

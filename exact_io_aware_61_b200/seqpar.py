@@ -23,6 +23,12 @@ sequence across ``W`` ranks:
 * **Merge.** ``fa_merge_partials`` combines the ``W`` blocks of every query
   row with the rescale rule. Only K/V cross the links; Q, O and the partial
   results stay on their rank.
+* **Backward.** The same ring. Each rank prepares its own rows once (D from
+  its O and dO, the merged LSE of its whole rows). At each step it adds the
+  visiting key block's share of dK and dV into f32 accumulators that travel
+  with that block, and its share of dQ into the rank's own accumulator
+  (``fa_bwd_partial``). After the last step the accumulators are back at the
+  ranks that own the keys.
 
 The exchange uses ``torch.distributed`` point-to-point operations (NCCL over
 NVLink on GPUs; any backend for the host logic). Every step of the attention
@@ -135,3 +141,88 @@ def ring_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool
             cur_k, cur_v = recv[t % 2]
     merge(o_parts, lse_parts, o, lse)
     return o, lse
+
+
+class LibraryBackwardOps:
+    """The CUDA calls of :func:`ring_backward` for one rank: ``fa_bwd_prep``,
+    ``fa_bwd_partial`` per key block, ``fa_bwd_dq``, ``fa_f32_to_bf16``."""
+
+    def __init__(self, q, k, causal: bool, scale: float, stream=None):
+        B, Hq, n, d = q.shape
+        self.Hkv = k.shape[1]
+        self.causal, self.scale, self.stream = causal, scale, stream
+        self.ws = torch.empty(max(_lib.fa_bwd_workspace_size(B, Hq, self.Hkv, n, d), 16), dtype=torch.uint8,
+                              device=q.device)
+
+    def prep(self, o, lse, do):
+        _lib.fa_bwd_prep(o, lse, do, self.ws, self.Hkv, self.stream)
+
+    def block(self, q, k, v, do, dk_acc, dv_acc, diag_offset: int):
+        _lib.fa_bwd_partial(q, k, v, do, dk_acc, dv_acc, self.ws, self.causal, self.scale, diag_offset, self.stream)
+
+    def finish(self, dq):
+        _lib.fa_bwd_dq(dq, self.ws, self.Hkv, self.stream)
+
+    def to_bf16(self, src, dst):
+        _lib.fa_f32_to_bf16(src, dst, self.stream)
+
+
+def ring_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                  do: torch.Tensor, causal: bool = False, scale: Optional[float] = None, group=None, *,
+                  ops=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients of :func:`ring_forward` for this rank's striped shards.
+
+    ``o`` and ``lse`` are this rank's rows of the forward (``ring_forward``'s
+    results: the merged, whole-row values), ``do`` the upstream gradient of
+    ``o``. Returns this rank's rows of ``(dQ, dK, dV)``, shaped like ``q``,
+    ``k``, ``v``. Collective over ``group``, like :func:`ring_forward`.
+    """
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    ops = ops or LibraryBackwardOps(q, k, causal, scale)
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    ops.prep(o, lse, do)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    acc = (torch.zeros(k.shape, dtype=torch.float32, device=k.device),
+           torch.zeros(v.shape, dtype=torch.float32, device=v.device))
+    if world == 1:
+        ops.block(q, k, v, do, acc[0], acc[1], 0)
+    else:
+        nxt = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
+        prv = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
+        kv_recv = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(2)]
+        acc_recv = [tuple(torch.empty_like(a) for a in acc) for _ in range(2)]
+        cur_k, cur_v = k, v
+        for t, (src, diag) in enumerate(ring_schedule(rank, world, causal)):
+            kv_reqs = []
+            if t + 1 < world:  # the next block's K, V travel while this one computes
+                nk, nv = kv_recv[t % 2]
+                kv_reqs = dist.batch_isend_irecv([
+                    dist.P2POp(dist.isend, cur_k, nxt, group),
+                    dist.P2POp(dist.isend, cur_v, nxt, group),
+                    dist.P2POp(dist.irecv, nk, prv, group),
+                    dist.P2POp(dist.irecv, nv, prv, group),
+                ])
+            ops.block(q, cur_k, cur_v, do, acc[0], acc[1], diag)
+            # this block's accumulators move on once this rank's share is in;
+            # the previous rank's (for the next block) arrive. After the last
+            # step each rank holds the accumulators of its own keys.
+            ndk, ndv = acc_recv[t % 2]
+            acc_reqs = dist.batch_isend_irecv([
+                dist.P2POp(dist.isend, acc[0], nxt, group),
+                dist.P2POp(dist.isend, acc[1], nxt, group),
+                dist.P2POp(dist.irecv, ndk, prv, group),
+                dist.P2POp(dist.irecv, ndv, prv, group),
+            ])
+            for req in kv_reqs + acc_reqs:
+                req.wait()
+            acc, acc_recv[t % 2] = (ndk, ndv), acc
+            if t + 1 < world:
+                cur_k, cur_v = kv_recv[t % 2]
+    ops.finish(dq)
+    ops.to_bf16(acc[0], dk)
+    ops.to_bf16(acc[1], dv)
+    return dq, dk, dv

@@ -287,6 +287,45 @@ FA_API int fa_bwd_noalloc(const void* q, const void* k, const void* v, const voi
                    int dtype, fa_stream_t stream);
 
 /*
+ * fa_bwd_partial -- one key block's share of the backward, for attention
+ * sharded over the sequence (the backward of fa_fwd_partial's blocks).
+ *
+ *   q, dO [B][Hq][N][d], k, v [B][Hkv][N][d]   inputs (bf16): this rank's
+ *                                               queries, a key block
+ *   dk_acc, dv_acc [B][Hkv][N][d]               float32 accumulators of the
+ *                                               key block's dK, dV: added to,
+ *                                               never cleared
+ *   workspace                                   as for fa_bwd, after
+ *                                               fa_bwd_prep on this rank's O,
+ *                                               dO and the LSE of its whole
+ *                                               rows (every key block); the
+ *                                               block's dQ is added into its
+ *                                               f32 dQ accumulator
+ *   diag_offset                                 as for fa_fwd_partial: with
+ *                                               causal = 1 query i sees key j
+ *                                               iff j <= i + diag_offset
+ * With the full rows' LSE and D, the block's weights are P = exp(scale S -
+ * LSE) and its share of the gradient is dQ += scale dS K, dK += scale dS^T Q,
+ * dV += P^T dO, dS = P (dP - D) ("The backward pass, and where the memory
+ * saving comes from"); summed over the key blocks it is fa_bwd's result.
+ * Call fa_bwd_prep once, fa_bwd_partial once per key block, then fa_bwd_dq
+ * for dQ and fa_f32_to_bf16 for dK and dV. dtype FA_BF16 with d in {64, 128};
+ * other cases return FA_ERR_UNSUPPORTED. Returns fa_status.
+ */
+FA_API int fa_bwd_partial(const void* q, const void* k, const void* v, const void* dO,
+                   float* dk_acc, float* dv_acc, void* workspace, size_t workspace_bytes,
+                   int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                   int diag_offset, int dtype, fa_stream_t stream);
+
+/*
+ * fa_f32_to_bf16 -- dst[i] = bf16(src[i]) (round to nearest even) for
+ * i < n; n a multiple of 4, both pointers 16-byte aligned device memory
+ * (FA_ERR_INVALID otherwise). For the dK, dV accumulators of
+ * fa_bwd_partial. Returns fa_status.
+ */
+FA_API int fa_f32_to_bf16(const float* src, void* dst, size_t n, fa_stream_t stream);
+
+/*
  * fa_bwd_varlen_workspace_size -- bytes of device workspace fa_bwd_varlen
  * needs: 4 * (2 * Hq * P + total_q * Hq * d + A), where P = the multiple
  * of 128 at or above 4 * ceil(total_q / 4) + 4 * batch + 128 (per query

@@ -1,4 +1,4 @@
-"""Parity of the sequence-sharding calls (fa_fwd_partial, fa_merge_partials) with the fp64 oracle.
+"""Parity of the sequence-sharding calls (fa_fwd_partial, fa_merge_partials, fa_bwd_partial) with the fp64 oracle.
 
 ``fa_fwd_partial`` is checked against ``attention_forward_positions`` with
 query i at position i + diag_offset and key j at position j, over offsets that
@@ -190,3 +190,96 @@ def test_striped_ring_emulated_w8_b2_h32_n8192_d128_sampled(fa):
         rows = sorted(set([0, 1, 7, 8, 9, N - 1] + [int(x) for x in rng.integers(0, N, 12)]))
         ro, rl = ORACLE.attention_forward_rows(qq, kk, vv, d ** -0.5, True, 0, 0, rows)
         _compare(INP.as_f64(o[b, h, rows]), INP.as_f64(lse[b, h, rows]), ro, rl)
+
+
+
+# --------------------------------------------------------------- backward
+
+GRAD_TOL = 2e-2
+
+
+def _rel(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-3 * np.sqrt(b.size), 1e-30))
+
+
+def test_bwd_partial_one_block_is_fa_bwd(fa):
+    """One block with offset 0 against zeroed accumulators is fa_bwd: dK, dV
+    bit for bit (head split 1), dQ to the rounding of its atomic order."""
+    B, Hq, Hkv, N, d = 2, 8, 4, 1000, 128
+    inp = INP.make_inputs(B, Hq, Hkv, N, d, "bf16", seed=91, grad=True)
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.forward(q, k, v, True)
+    dq_ref, dk_ref, dv_ref = fa.backward(q, k, v, o, lse, do, True)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, Hq, Hkv, N, d), dtype=torch.uint8, device="cuda")
+    gk = Guarded(k.shape, torch.float32, fill=0.0)
+    gv = Guarded(v.shape, torch.float32, fill=0.0)
+    fa.fa_bwd_prep(o, lse, do, ws, Hkv)
+    fa.fa_bwd_partial(q, k, v, do, gk.t, gv.t, ws, True, d ** -0.5, 0)
+    dq = torch.empty_like(q)
+    fa.fa_bwd_dq(dq, ws, Hkv)
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    fa.fa_f32_to_bf16(gk.t, dk)
+    fa.fa_f32_to_bf16(gv.t, dv)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.FA_OK
+    check_all(("dK acc", gk), ("dV acc", gv))
+    assert torch.equal(dk, dk_ref) and torch.equal(dv, dv_ref)
+    diff = (dq.float() - dq_ref.float()).abs()
+    assert torch.all(diff <= 2.0 ** -7 * dq_ref.float().abs() + 1e-6)
+
+
+def _emulate_ring_backward(fa, q, k, v, do, world, causal, scale):
+    """Every rank's ring backward on one GPU: the forward shards from the
+    emulated ring forward, then per rank its prep, one fa_bwd_partial per key
+    block (the accumulators of each key shard are shared, as if they had
+    travelled), its dQ; finally the accumulators to bf16."""
+    o, lse = _emulate_ring(fa, q, k, v, world, causal, scale)
+    shard = lambda t, r: seqpar.shard_striped(t, r, world)
+    ks = [shard(k, c) for c in range(world)]
+    vs = [shard(v, c) for c in range(world)]
+    acc_k = [torch.zeros(t.shape, dtype=torch.float32, device="cuda") for t in ks]
+    acc_v = [torch.zeros(t.shape, dtype=torch.float32, device="cuda") for t in vs]
+    dqs = []
+    for r in range(world):
+        qr, dor = shard(q, r), shard(do, r)
+        ops = seqpar.LibraryBackwardOps(qr, ks[r], causal, scale)
+        ops.prep(shard(o, r), seqpar.shard_striped(lse[..., None], r, world)[..., 0].contiguous(), dor)
+        for src, diag in seqpar.ring_schedule(r, world, causal):
+            ops.block(qr, ks[src], vs[src], dor, acc_k[src], acc_v[src], diag)
+        dq = torch.empty_like(qr)
+        ops.finish(dq)
+        dqs.append(dq)
+    dks = [torch.empty_like(t) for t in ks]
+    dvs = [torch.empty_like(t) for t in vs]
+    for c in range(world):
+        fa.fa_f32_to_bf16(acc_k[c], dks[c])
+        fa.fa_f32_to_bf16(acc_v[c], dvs[c])
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_status() == fa.FA_OK
+    return tuple(seqpar.unshard_striped(x) for x in (dqs, dks, dvs))
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+@pytest.mark.parametrize("causal", [True, False])
+def test_striped_ring_backward_emulated_equals_unsharded(fa, world, causal):
+    B, Hq, Hkv, d = 1, 4, 2, 128
+    N = {2: 770, 3: 771, 4: 772}[world]
+    inp = INP.make_inputs(B, Hq, Hkv, N, d, "bf16", seed=29 + world, grad=True)
+    q, k, v, do = (inp[n].cuda().contiguous() for n in ("q", "k", "v", "do"))
+    dq, dk, dv = _emulate_ring_backward(fa, q, k, v, do, world, causal, d ** -0.5)
+    rq, rk, rv, _ = ORACLE.attention_backward(*(INP.as_f64(inp[n]) for n in ("q", "k", "v", "do")), d ** -0.5, causal)
+    assert _rel(INP.as_f64(dq), rq) <= GRAD_TOL
+    assert _rel(INP.as_f64(dk), rk) <= GRAD_TOL
+    assert _rel(INP.as_f64(dv), rv) <= GRAD_TOL
+
+
+def test_striped_ring_backward_emulated_w4_d64_gqa(fa):
+    B, Hq, Hkv, N, d, world = 2, 8, 2, 2048, 64, 4
+    inp = INP.make_inputs(B, Hq, Hkv, N, d, "bf16", seed=4242, grad=True)
+    q, k, v, do = (inp[n].cuda().contiguous() for n in ("q", "k", "v", "do"))
+    dq, dk, dv = _emulate_ring_backward(fa, q, k, v, do, world, True, d ** -0.5)
+    rq, rk, rv, _ = ORACLE.attention_backward(*(INP.as_f64(inp[n]) for n in ("q", "k", "v", "do")), d ** -0.5, True)
+    assert _rel(INP.as_f64(dq), rq) <= GRAD_TOL
+    assert _rel(INP.as_f64(dk), rk) <= GRAD_TOL
+    assert _rel(INP.as_f64(dv), rv) <= GRAD_TOL

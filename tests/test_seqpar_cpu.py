@@ -1,9 +1,10 @@
-"""Host logic of the sequence-sharded forward (striped tokens, K/V ring, merge) on CPU.
+"""Host logic of the sequence-sharded forward and backward (striped tokens, K/V ring) on CPU.
 
-The ring schedule, the diagonal offsets and the point-to-point exchange of
-``exact_io_aware_61_b200.seqpar.ring_forward`` run here over gloo ranks, with
-the fp64 oracle standing in for the two CUDA calls (the block forward and the
-merge); the gathered result must equal the oracle's attention over the whole,
+The ring schedule, the diagonal offsets and the point-to-point exchanges of
+``exact_io_aware_61_b200.seqpar.ring_forward`` and ``ring_backward`` run here
+over gloo ranks, with the fp64 oracle standing in for the CUDA calls (block
+forward and merge; preprocess, block backward, dQ conversion); the gathered
+results must equal the oracle's attention and gradients over the whole,
 unsharded sequence. The CUDA calls themselves are checked on the GPU.
 """
 
@@ -107,3 +108,66 @@ def test_striped_shards_round_trip():
     assert torch.equal(seqpar.striped_positions(3, 1, 4), torch.tensor([1, 5, 9]))
     with pytest.raises(ValueError):
         seqpar.shard_striped(x, 0, 5)
+
+
+class OracleBackwardOps:
+    """The fp64 oracle in place of fa_bwd_prep / fa_bwd_partial / fa_bwd_dq / fa_f32_to_bf16."""
+
+    def __init__(self, causal, scale):
+        self.causal, self.scale = causal, scale
+
+    def prep(self, o, lse, do):
+        self.lse = lse.double().numpy()
+        self.D = np.sum(do.double().numpy() * o.double().numpy(), axis=-1)
+        self.dq = None
+
+    def block(self, q, k, v, do, dk_acc, dv_acc, diag_offset):
+        n = q.shape[2]
+        bq, bk, bv = ORACLE.attention_backward_block(q.numpy(), k.numpy(), v.numpy(), do.numpy(), self.lse, self.D,
+                                                     np.arange(n) + diag_offset, np.arange(n), self.scale, self.causal)
+        self.dq = bq if self.dq is None else self.dq + bq
+        dk_acc += torch.from_numpy(bk).to(dk_acc.dtype)
+        dv_acc += torch.from_numpy(bv).to(dv_acc.dtype)
+
+    def finish(self, dq):
+        dq.copy_(torch.from_numpy(self.dq))
+
+    def to_bf16(self, src, dst):
+        dst.copy_(src)
+
+
+def _ring_bwd_worker(rank, world, port, causal, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        inp = INP.make_inputs(SHAPE["B"], SHAPE["Hq"], SHAPE["Hkv"], SHAPE["N"], SHAPE["d"], "f32", seed=137,
+                              grad=True)
+        q, k, v, do = (inp[n].double() for n in ("q", "k", "v", "do"))
+        o, lse = ORACLE.attention_forward(q.numpy(), k.numpy(), v.numpy(), 0.37, causal)
+        sh = lambda t: seqpar.shard_striped(t, rank, world)
+        # the dK/dV accumulators are f32, as the library's; dQ and the exchange of K, V in f64
+        o_r = sh(torch.from_numpy(o))
+        lse_r = sh(torch.from_numpy(lse)[..., None])[..., 0]
+        dq, dk, dv = seqpar.ring_backward(sh(q), sh(k), sh(v), o_r, lse_r, sh(do), causal=causal, scale=0.37,
+                                          ops=OracleBackwardOps(causal, 0.37))
+        out[rank] = tuple(t.numpy().tolist() for t in (dq, dk, dv))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ring_backward_equals_unsharded_gradients_gloo(world, causal):
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_ring_bwd_worker, args=(world, port, causal, out), nprocs=world, join=True)
+        res = dict(out)
+    inp = INP.make_inputs(SHAPE["B"], SHAPE["Hq"], SHAPE["Hkv"], SHAPE["N"], SHAPE["d"], "f32", seed=137, grad=True)
+    q, k, v, do = (INP.as_f64(inp[n]) for n in ("q", "k", "v", "do"))
+    rq, rk, rv, _ = ORACLE.attention_backward(q, k, v, do, 0.37, causal)
+    for i, ref in enumerate((rq, rk, rv)):
+        got = seqpar.unshard_striped([torch.tensor(res[r][i]) for r in range(world)]).numpy()
+        # dK, dV accumulate in float32 across the ring
+        assert np.max(np.abs(got - ref)) < 1e-5 * max(1.0, np.max(np.abs(ref)))
