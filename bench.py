@@ -643,7 +643,7 @@ def run_fwd_shape(args, rank, world, local):
 
 
 def run_seqpar(args, rank, world, local):
-    """Time the sequence-sharded causal forward (striped tokens, K/V ring, merge).
+    """Time the sequence-sharded causal forward (striped tokens, K/V ring, merge) and its backward.
 
     On one GPU the W ranks' work is emulated: the busiest rank's W blocks
     (``fa_fwd_partial`` against every rank's K/V shard, all held on this GPU)
@@ -744,6 +744,47 @@ def run_seqpar(args, rank, world, local):
         "pct_of_peak": round(100 * tflops / peaks["bf16_tflops"], 2), "peak_note": f"{src} bf16 GEMM (burst)",
         "clocks": clocks,
     }
+    # the backward of the same rank: prep, one fa_bwd_partial per block, dQ
+    # and (for the keys the rank owns) dK, dV conversions; under
+    # torch.distributed the whole ring_backward with its exchanges
+    g.manual_seed(SEED + 7 + rank)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+    if world == 1:
+        bops = seqpar.LibraryBackwardOps(q, kv[0][0], True, scale, stream)
+        accs = [(torch.zeros(kv[0][0].shape, dtype=torch.float32, device=dev),
+                 torch.zeros(kv[0][1].shape, dtype=torch.float32, device=dev)) for _ in range(W)]
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(kv[0][0]), torch.empty_like(kv[0][1])
+    else:
+        o, lse = seqpar.ring_forward(q, k, v, causal=True, scale=scale)
+
+    def run_bwd():
+        if world > 1:
+            seqpar.ring_backward(q, k, v, o, lse, do, causal=True, scale=scale)
+            return
+        bops.prep(o, lse, do)
+        for src, diag in sched:
+            bops.block(q, kv[src][0], kv[src][1], do, accs[src][0], accs[src][1], diag)
+        bops.finish(dq)
+        bops.to_bf16(accs[me][0], dk)
+        bops.to_bf16(accs[me][1], dv)
+
+    for _ in range(args.warmup):
+        run_bwd()
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for _ in range(args.steps):
+        run_bwd()
+    b1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    if fa.fa_last_device_status(stream) != fa.FA_OK:
+        raise RuntimeError("device status reports a timeout")
+    bwd_ms = max_over_ranks(b0.elapsed_time(b1) / args.steps, world, dev)
+    out["bwd"] = {"ms_per_step": round(bwd_ms, 4), "tflops": round(2.5 * flops / bwd_ms / 1e9, 2),
+                  "pct_of_peak": round(100 * 2.5 * flops / bwd_ms / 1e9 / peaks["bf16_tflops"], 2),
+                  "flops_note": "2.5 x the rank's forward FLOPs (the usual backward convention)"}
     if world == 1:
         blk = [a.elapsed_time(b) for kind, (a, b) in blk_ev if kind == "block"]
         mrg = [a.elapsed_time(b) for kind, (a, b) in blk_ev if kind == "merge"]
