@@ -50,8 +50,8 @@ SPEC_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor peak, vendor figure (context
 PROFILED = {
     # ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum,
     #     sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active at the benchmark shape
-    "bwd_main": {"src": "22cb3aa90e626389", "dram_bytes": 825_633_792 + 499_321_344, "tensor_pipe_active_pct": 41.89},
-    "fwd": {"src": "22cb3aa90e626389", "dram_bytes": 403_091_456 + 116_115_712, "tensor_pipe_active_pct": 50.53},
+    "bwd_main": {"src": "4a118df09958197f", "dram_bytes": 826_841_088 + 499_585_024, "tensor_pipe_active_pct": 41.80},
+    "fwd": {"src": "4a118df09958197f", "dram_bytes": 403_137_536 + 115_962_880, "tensor_pipe_active_pct": 50.90},
 }
 
 
