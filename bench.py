@@ -805,6 +805,88 @@ def run_seqpar(args, rank, world, local):
         dist.destroy_process_group()
 
 
+def varlen_lengths(total: int, lo: int, hi: int, seed: int):
+    """Seeded sequence lengths, uniform in [lo, hi], the last one cut so that they sum to ``total``."""
+    import random
+
+    rng = random.Random(seed)
+    lens = []
+    while sum(lens) < total:
+        lens.append(min(rng.randint(lo, hi), total - sum(lens)))
+    return lens
+
+
+def run_varlen(args, rank, world, local):
+    """Time fa_fwd_varlen and fa_bwd_varlen on one GPU over a packed batch of
+    sequences of mixed lengths (causal, each sequence's queries against its
+    own keys). FLOPs: per sequence 4 * Hq * L * (L + 1) / 2 * d forward (its
+    visible pairs), 2.5 times that backward."""
+    import torch
+
+    import exact_io_aware_61_b200 as fa
+    from exact_io_aware_61_b200 import inputs as inp_mod
+
+    if world != 1:
+        raise SystemExit("--varlen runs on one GPU")
+    total, lo, hi, Hq, Hkv, d = (int(x) for x in args.varlen.split(","))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fa.load()
+    lens = varlen_lengths(total, lo, hi, SEED)
+    host = inp_mod.make_varlen_inputs(lens, lens, Hq, Hkv, d, "bf16", SEED, grad=True)
+    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
+    cu = host["cu_q"].to(dev)
+    scale = d ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(fa.fa_bwd_varlen_workspace_size(len(lens), total, total, Hq, Hkv, d), 16),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    mx = max(lens)
+
+    def fwd():
+        fa.fa_fwd_varlen(q, k, v, o, lse, cu, cu, mx, True, scale, stream)
+
+    def bwd():
+        fa.fa_bwd_varlen(q, k, v, o, lse, do, dq, dk, dv, cu, cu, mx, mx, ws, True, scale, stream)
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(physical_gpu_index(local))
+    sampler.start()
+    for e0, e1, e2 in ev:
+        e0.record(stream)
+        fwd()
+        e1.record(stream)
+        bwd()
+        e2.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if fa.fa_last_device_status(stream) != fa.FA_OK:
+        raise RuntimeError("device status reports an error")
+    f_ms = statistics.median(a.elapsed_time(b) for a, b, _ in ev)
+    b_ms = statistics.median(b.elapsed_time(c) for _, b, c in ev)
+    fflops = sum(4.0 * Hq * L * (L + 1) / 2 * d for L in lens)
+    peaks, src = load_peaks()
+    f_tf, b_tf = fflops / f_ms / 1e9, 2.5 * fflops / b_ms / 1e9
+    print(json.dumps({
+        "metric": "variable-length causal attention fwd+bwd TFLOP/s", "value": round(3.5 * fflops / (f_ms + b_ms) / 1e9, 2),
+        "unit": "TFLOP/s", "higher_is_better": True, "steps": args.steps, "warmup": args.warmup,
+        "fwd_tflops": round(f_tf, 2), "bwd_tflops": round(b_tf, 2), "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4),
+        "pct_of_peak": {"fwd": round(100 * f_tf / peaks["bf16_tflops"], 2),
+                        "bwd": round(100 * b_tf / peaks["bf16_tflops"], 2)},
+        "peak_note": f"{src} bf16 GEMM (burst)",
+        "config": {"workload": f"causal bf16 packed batch of {len(lens)} sequences, {total} tokens, lengths uniform "
+                               f"in [{lo}, {hi}] (seeded), Hq={Hq} Hkv={Hkv} d={d}",
+                   "lengths": lens, "l2": "no flush: Q, K, V and the gradients exceed the L2"},
+        "clocks": clocks, "dtype": "bf16", "data": "synthetic: i.i.d. N(0,1), seeded"}))
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return  # rank 0 alone times the oracle; the others exit without work
@@ -858,6 +940,8 @@ def main(argv=None):
                     help="B,Hq,Hkv,Nq,Nk,d: time the KV-cache (decode) forward instead of the benchmark step")
     ap.add_argument("--seqpar", default=None,
                     help="B,Hq,Hkv,N,d,W: time the sequence-sharded causal forward over W striped ranks")
+    ap.add_argument("--varlen", default=None,
+                    help="total,lo,hi,Hq,Hkv,d: time the variable-length forward and backward on a packed batch")
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d of a smaller case for profiling (default: the benchmark workload)")
     args = ap.parse_args(argv)
@@ -874,6 +958,8 @@ def main(argv=None):
             ap.error(f"--gpus {args.gpus} needs a launch with torch.distributed.run (one rank per GPU)")
     if args.seqpar:
         run_seqpar(args, rank, world, local)
+    elif args.varlen:
+        run_varlen(args, rank, world, local)
     elif args.kvcache:
         run_kvcache(args, rank, world, local)
     elif args.fwd:
