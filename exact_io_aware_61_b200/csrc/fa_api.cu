@@ -295,30 +295,46 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
   return launch_status(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_2tile_kernel<HD, true>));
 }
 
-template <int HD, int UNROLL>
-int launch_merge_u(const void* o_parts, const float* lse_parts, int n_parts, long long rows, void* o, float* lse,
-                   int num_sms, cudaStream_t stream) {
-  constexpr int TPR = HD / 8;
-  const long long threads = rows * TPR;
-  const long long want = (threads + fa::MergeCfg::THREADS - 1) / fa::MergeCfg::THREADS;
-  // grid-stride over rows with exactly the blocks that are resident at once
-  // (a second, partial wave would leave its blocks a full share of rows)
+// The merge's grid: grid-stride over rows with exactly the blocks that are
+// resident at once (a second, partial wave would leave its blocks a full share
+// of rows). Planned before any launch, since it queries the runtime.
+struct MergePlan {
+  int unroll;  // parts whose loads are in flight together: 4 or 8
+  unsigned blocks;
+};
+
+template <int HD>
+int plan_merge(int n_parts, long long rows, int num_sms, MergePlan* mp) {
+  mp->unroll = n_parts <= 4 ? 4 : 8;
+  const long long want = (rows * (HD / 8) + fa::MergeCfg::THREADS - 1) / fa::MergeCfg::THREADS;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fa::fa_merge_partials_kernel<HD, UNROLL>,
-                                                    fa::MergeCfg::THREADS, 0) != cudaSuccess ||
-      per_sm < 1)
-    return FA_ERR_CUDA;
-  const long long blocks = std::min<long long>(want, static_cast<long long>(per_sm) * num_sms);
-  fa::fa_merge_partials_kernel<HD, UNROLL><<<static_cast<unsigned>(blocks), fa::MergeCfg::THREADS, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o_parts), lse_parts, n_parts, rows, static_cast<__nv_bfloat16*>(o), lse);
-  return launch_status();
+  const cudaError_t e =
+      mp->unroll == 4
+          ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fa::fa_merge_partials_kernel<HD, 4>,
+                                                          fa::MergeCfg::THREADS, 0)
+          : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fa::fa_merge_partials_kernel<HD, 8>,
+                                                          fa::MergeCfg::THREADS, 0);
+  if (e != cudaSuccess || per_sm < 1) return FA_ERR_CUDA;
+  mp->blocks = static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(per_sm) * num_sms));
+  return FA_OK;
 }
 
 template <int HD>
-int launch_merge(const void* o_parts, const float* lse_parts, int n_parts, long long rows, void* o, float* lse,
-                 int num_sms, cudaStream_t stream) {
-  return n_parts <= 4 ? launch_merge_u<HD, 4>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, stream)
-                      : launch_merge_u<HD, 8>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, stream);
+int launch_merge(const MergePlan& mp, const void* o_parts, const float* lse_parts, int n_parts, long long rows,
+                 void* o, float* lse, cudaStream_t stream) {
+  const auto* src = static_cast<const __nv_bfloat16*>(o_parts);
+  auto* dst = static_cast<__nv_bfloat16*>(o);
+  if (mp.unroll == 4)
+    fa::fa_merge_partials_kernel<HD, 4><<<mp.blocks, fa::MergeCfg::THREADS, 0, stream>>>(src, lse_parts, n_parts,
+                                                                                        rows, dst, lse);
+  else
+    fa::fa_merge_partials_kernel<HD, 8><<<mp.blocks, fa::MergeCfg::THREADS, 0, stream>>>(src, lse_parts, n_parts,
+                                                                                        rows, dst, lse);
+  return launch_status();
+}
+
+int num_sms_of(int dev, int* num_sms) {
+  return cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 template <int HD>
@@ -771,14 +787,16 @@ int launch_decode_tc(const void* q, const void* k, const void* v, void* o, float
   p.splits = tp.S;
   p.split_tiles = tp.split_tiles;
   p.rows_total = static_cast<int>(rows_total);
+  MergePlan mplan{};
+  if (tp.S > 1) {  // everything that can fail short of a launch, before the first launch
+    int dev = 0, num_sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || num_sms_of(dev, &num_sms) != FA_OK) return FA_ERR_CUDA;
+    if ((rc = plan_merge<HD>(tp.S, rows_total, num_sms, &mplan)) != FA_OK) return rc;
+  }
   fa::fa_fwd_bf16_kernel<HD, true><<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   if (launch_status(reinterpret_cast<const void*>(&fa::fa_fwd_bf16_kernel<HD, true>)) != FA_OK) return FA_ERR_CUDA;
   if (tp.S == 1) return FA_OK;
-  int dev = 0, num_sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return FA_ERR_CUDA;
-  return launch_merge<HD>(o_part, lse_part, tp.S, rows_total, o, lse, num_sms, stream);
+  return launch_merge<HD>(mplan, o_part, lse_part, tp.S, rows_total, o, lse, stream);
 }
 
 // Checks shared by the backward entry points. `ptrs` must all be 16-byte aligned and non-null.
@@ -913,12 +931,19 @@ int fa_merge_partials(const void* o_parts, const float* lse_parts, int n_parts, 
   if (rc != FA_OK) return rc;
   if ((rc = prepare_kernels(dev)) != FA_OK) return rc;
   int num_sms = 0;
-  if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FA_ERR_CUDA;
+  if ((rc = num_sms_of(dev, &num_sms)) != FA_OK) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MergePlan mp{};
   switch (d) {
-    case 64: return launch_merge<64>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
-    case 128: return launch_merge<128>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
-    default: return launch_merge<256>(o_parts, lse_parts, n_parts, rows, o, lse, num_sms, s);
+    case 64:
+      if ((rc = plan_merge<64>(n_parts, rows, num_sms, &mp)) != FA_OK) return rc;
+      return launch_merge<64>(mp, o_parts, lse_parts, n_parts, rows, o, lse, s);
+    case 128:
+      if ((rc = plan_merge<128>(n_parts, rows, num_sms, &mp)) != FA_OK) return rc;
+      return launch_merge<128>(mp, o_parts, lse_parts, n_parts, rows, o, lse, s);
+    default:
+      if ((rc = plan_merge<256>(n_parts, rows, num_sms, &mp)) != FA_OK) return rc;
+      return launch_merge<256>(mp, o_parts, lse_parts, n_parts, rows, o, lse, s);
   }
 }
 
