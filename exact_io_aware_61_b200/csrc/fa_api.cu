@@ -950,11 +950,13 @@ int fa_merge_partials(const void* o_parts, const float* lse_parts, int n_parts, 
 int fa_bwd_partial(const void* q, const void* k, const void* v, const void* dO, float* dk_acc, float* dv_acc,
                    void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
                    int causal, int diag_offset, int dtype, fa_stream_t stream) {
+  int rc = check_shape(B, Hq, Hkv, N, d, scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (dtype != FA_BF16 || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
   int dev = 0;
-  int rc = check_bwd({q, k, v, dO, dk_acc, dv_acc}, workspace, workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype,
-                     &dev);
+  rc = check_bwd({q, k, v, dO, dk_acc, dv_acc}, workspace, workspace_bytes, B, Hq, Hkv, N, d, scale, causal, dtype,
+                 &dev);
   if (rc != FA_OK) return rc < 0 ? FA_OK : rc;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   // offsets beyond +-N change nothing; clamping keeps the kernel's index sums in range
   const int shift = causal ? std::max(-N, std::min(N, diag_offset)) : 0;
   BwdPlan pl;

@@ -196,3 +196,30 @@ def test_varlen_validation_before_any_device_work(lib):
     assert call(cu=66) == fa.FA_ERR_INVALID           # misaligned offsets
     assert call(cu=0) == fa.FA_ERR_INVALID            # no offsets
     assert call(batch=0) == fa.FA_OK and call(tq=0, max_q=0) == fa.FA_OK  # empty
+
+
+def test_sequence_sharding_calls_validate_before_any_device_work(lib):
+    p, m = ctypes.c_void_p(64), ctypes.c_void_p(66)
+    # fa_fwd_partial: fp32 and bad sizes
+    assert lib.fa_fwd_partial(p, p, p, p, p, 1, 2, 2, 8, 64, 0.1, 1, -1, 1, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_partial(p, p, p, p, p, 1, 3, 2, 8, 64, 0.1, 1, -1, 0, None) == fa.FA_ERR_INVALID
+    assert lib.fa_fwd_partial(p, p, p, p, p, 0, 2, 2, 8, 64, 0.1, 1, -1, 0, None) == fa.FA_OK  # empty
+    # fa_merge_partials: sizes, head dimension, overlap of output and input, alignment
+    assert lib.fa_merge_partials(p, p, 0, 16, ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 21), 64, 0, None) \
+        == fa.FA_ERR_INVALID
+    assert lib.fa_merge_partials(p, p, 2, 16, ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 21), 96, 0, None) \
+        == fa.FA_ERR_INVALID
+    assert lib.fa_merge_partials(ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 22), 2, 16, ctypes.c_void_p(1 << 20),
+                                 ctypes.c_void_p(1 << 23), 64, 0, None) == fa.FA_ERR_INVALID   # o is part 0
+    assert lib.fa_merge_partials(m, p, 2, 16, ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 21), 64, 0, None) \
+        == fa.FA_ERR_INVALID
+    assert lib.fa_merge_partials(p, p, 2, 0, p, p, 64, 0, None) == fa.FA_OK  # no rows
+    # fa_bwd_partial: d = 256 and fp32 are not implemented; short workspace
+    args = [p] * 6
+    assert lib.fa_bwd_partial(*args, p, 1 << 30, 1, 2, 2, 8, 256, 0.1, 1, -1, 0, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_bwd_partial(*args, p, 1 << 30, 1, 2, 2, 8, 64, 0.1, 1, -1, 1, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_bwd_partial(*args, p, 16, 1, 2, 2, 8, 64, 0.1, 1, -1, 0, None) == fa.FA_ERR_WORKSPACE
+    # fa_f32_to_bf16: a count that is not a multiple of 4, misaligned pointers
+    assert lib.fa_f32_to_bf16(p, p, 6, None) == fa.FA_ERR_INVALID
+    assert lib.fa_f32_to_bf16(m, p, 8, None) == fa.FA_ERR_INVALID
+    assert lib.fa_f32_to_bf16(p, p, 0, None) == fa.FA_OK
