@@ -28,9 +28,10 @@
 //               owns key columns [32h, 32h + 32): P (bf16) and dS (bf16)
 //               into 128-byte-swizzled shared tiles [query][key], which are
 //               the B operands of dV^T and dK^T and the A operand of dQ
-//   warps 8-11  dQ drain: thread = query row; loads a 128-column half of dQ
-//               from TMEM, frees it, then adds it into the f32 accumulator
-//               (red.global.add.v4.f32)
+//   warps 8-11  dQ drain: loads dQ from TMEM in 64-column pieces (16x256b
+//               shape), frees each as far as the next MMA needs it, and adds
+//               it into the f32 accumulator, each warp-wide reduction 256
+//               contiguous bytes of one row
 //   warp 12     TMA producer; warp 13 TMEM allocator and MMA issuer
 // Per step (query tile t) the issuer runs S, dP, dV^T (once P is in shared
 // memory), dK^T (once dS is), dQ half 1, dQ half 0.
@@ -38,6 +39,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <utility>
+
 #include "sm100_ptx.cuh"
 
 namespace fa {
@@ -63,7 +66,7 @@ struct Bwd256Cfg {
   static constexpr int OTHER_REGS = 96;
   static_assert(128 * (2 * COMPUTE_REGS + DRAIN_REGS + OTHER_REGS) <= THREADS * LAUNCH_REGS,
                 "register split exceeds the launch allocation");
-  static constexpr int KV_GROUP = 8;             // (batch, KV head) pairs scheduled together
+  static constexpr int KV_GROUP = 4;             // (batch, KV head) pairs scheduled together (their working set stays in L2)
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_DV = 0, T_DK = 128, T_S = 256, T_DP = 320, T_DQ0 = 384, T_DQ1 = 256;
 };
@@ -84,6 +87,47 @@ struct Bwd256Params {
   unsigned long long timeout_ns;
 };
 
+// The dQ drain's reductions of one set of 8 rows (RB .. RB + 7 of the warp's 32)
+// over a 64-column piece. On entry lane 4 g + c holds, in x[k], columns
+// 8k + 2c, 8k + 2c + 1 of row RB + g (k = 0..7: the 16x256b layout). An 8 x 8
+// transpose over the lane groups g (three butterfly stages of XOR shuffles;
+// the register indices stay compile-time constants) leaves in x[j] columns
+// 8g + 2c, 8g + 2c + 1 of row RB + j, so that each reduction instruction of
+// the warp covers 256 contiguous bytes of one row (whole lines: L2 takes
+// those about 1.7 times faster than 32-byte pieces of 8 rows).
+// x[J] (row RB + J, 1 KB per row of 256 floats) into the accumulator, the
+// row offset an immediate of the instruction
+template <int RB, int J>
+FA_DEV void drain_red(float* base, const float (&x)[8][2], int live) {
+  if (RB + J < live) red_add_v2_f32<(RB + J) * Bwd256Cfg::HD * 4>(base, x[J][0], x[J][1]);
+}
+
+template <int RB, size_t... J>
+FA_DEV void drain_reds(float* base, const float (&x)[8][2], int live, std::index_sequence<J...>) {
+  (drain_red<RB, static_cast<int>(J)>(base, x, live), ...);
+}
+
+template <int RB>
+FA_DEV void drain_rowset(float* base, float (&x)[8][2], int g, int live) {
+#pragma unroll
+  for (int s = 0; s < 3; ++s) {
+    const int m = 1 << s;
+    const bool hi = (g & m) != 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k & m) continue;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float send = hi ? x[k][e] : x[k | m][e];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 4 * m);
+        if (hi) x[k][e] = recv;
+        else x[k | m][e] = recv;
+      }
+    }
+  }
+  drain_reds<RB>(base, x, live, std::make_index_sequence<8>{});
+}
+
 // 16 warps, 4 per SM sub-partition: 16384 / 128 -> 128 registers at launch.
 __global__ void __launch_bounds__(512, 1)
     fa_bwd256_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -93,7 +137,7 @@ __global__ void __launch_bounds__(512, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_kv, bar_qfull, bar_qempty, bar_dofull, bar_doempty, bar_sfull, bar_dpfull;
   __shared__ uint64_t bar_pfull, bar_pempty, bar_dsfull, bar_dsempty;
-  __shared__ uint64_t bar_dq0full, bar_dq1full, bar_dq0free, bar_dq1free, bar_final;
+  __shared__ uint64_t bar_dq0full, bar_dq1full, bar_dq0free, bar_dq1afree, bar_dq1bfree, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -150,7 +194,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(smem_u32(&bar_pfull), 256);
     mbar_init(smem_u32(&bar_dsfull), 256);
     mbar_init(smem_u32(&bar_dq0free), 128);
-    mbar_init(smem_u32(&bar_dq1free), 128);
+    mbar_init(smem_u32(&bar_dq1afree), 128);
+    mbar_init(smem_u32(&bar_dq1bfree), 128);
     fence_mbar_init();
   }
   if (warp == 13) {
@@ -213,17 +258,18 @@ __global__ void __launch_bounds__(512, 1)
       for (int t = 0; ok && t < steps; ++t) {
         const uint32_t ph = t & 1;
         // S = Q K^T over d: the S columns are free once the drain has read
-        // dQ(t-1) half 1 from them
+        // the first 64 columns of dQ(t-1) half 1 from them
         if (!mbar_wait(smem_u32(&bar_qfull), ph, wc)) { ok = false; break; }
-        if (t > 0 && !mbar_wait(smem_u32(&bar_dq1free), ph ^ 1, wc)) { ok = false; break; }
+        if (t > 0 && !mbar_wait(smem_u32(&bar_dq1afree), ph ^ 1, wc)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 16; ++kk)
           mma_bf16_ss(tmem + C::T_S, sdesc_sw128(sQ + (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32, 16, 1024),
                       sdesc_sw128(sK + (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
         mma_commit(smem_u32(&bar_sfull));
-        // dP = dO V^T
+        // dP = dO V^T, in the columns of dQ(t-1) half 1's last 64
         if (!mbar_wait(smem_u32(&bar_dofull), ph, wc)) { ok = false; break; }
+        if (t > 0 && !mbar_wait(smem_u32(&bar_dq1bfree), ph ^ 1, wc)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 16; ++kk)
@@ -369,46 +415,63 @@ __global__ void __launch_bounds__(512, 1)
   } else {
     set_max_regs<C::DRAIN_REGS, C::LAUNCH_REGS>();
     // ------------------------------------------------------------ dQ drain
-    // Thread = query row r. Per half (half 1 first, in the order the MMAs
-    // produce them): the whole 128-column half is loaded, its columns freed,
-    // then added into the f32 accumulator with 16-byte reductions.
-    const int r = threadIdx.x - 256;
+    // dQ(t) leaves TMEM in four 64-column pieces: half 1 first (in the order
+    // the MMAs produce the halves), and of it first the piece over the S
+    // columns, which S(t+1) waits for, then the piece over the dP columns.
+    // Each piece is loaded in the 16x256b shape (32 rows x 64 columns a warp),
+    // its columns freed as far as the next MMA needs them, transposed across
+    // the lanes (drain_rowset) and added into the f32 accumulator with 8-byte
+    // reductions, each warp instruction 256 contiguous bytes of one row.
     const uint32_t lane_base = ((warp & 3) * 32u) << 16;
+    const int wrow = (warp & 3) * 32;  // the warp's 32 rows of the tile
+    const int g = lane >> 2, c = lane & 3;
     bool ok = true;
     for (int t = 0; ok && t < steps; ++t) {
       int bhq, q0;
       step_tile(t, bhq, q0);
       const uint32_t ph = t & 1;
-      const bool live = q0 + r < p.N;
-      float* row = p.dq_acc + (static_cast<size_t>(bhq) * p.N + (live ? q0 + r : 0)) * C::HD;
+      float* tile = p.dq_acc + (static_cast<size_t>(bhq) * p.N + q0) * C::HD;
+      const int live = p.N - q0 - wrow;  // rows of the warp's 32 inside N
 #pragma unroll 1
-      for (int i = 0; i < 2; ++i) {
-        const int half = 1 - i;
-        if (!warp_wait(smem_u32(half == 0 ? &bar_dq0full : &bar_dq1full), ph, wc)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t src = tmem + lane_base + (half == 0 ? C::T_DQ0 : C::T_DQ1);
-        uint32_t v[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32_async(src + c * 32, v[c]);
-        tmem_wait_ld32(v[0]);
-#pragma unroll
-        for (int c = 1; c < 4; ++c) tmem_tie32(v[c]);
-        tc_fence_before();
-        mbar_arrive(smem_u32(half == 0 ? &bar_dq0free : &bar_dq1free));
-        if (live) {
-          float* dst = row + half * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int x = 0; x < 8; ++x)
-              red_add_v4_f32(dst + c * 32 + 4 * x, __uint_as_float(v[c][4 * x]), __uint_as_float(v[c][4 * x + 1]),
-                             __uint_as_float(v[c][4 * x + 2]), __uint_as_float(v[c][4 * x + 3]));
+      for (int i = 0; i < 4; ++i) {
+        const int half = i < 2 ? 1 : 0;
+        const int piece = i & 1;
+        if (piece == 0 && !warp_wait(smem_u32(half == 0 ? &bar_dq0full : &bar_dq1full), ph, wc)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t src = tmem + lane_base + (half == 0 ? C::T_DQ0 : C::T_DQ1) + piece * 64;
+        uint32_t va[32], vb[32];
+        tmem_ld_16x256b_x8_async(src, va);                // rows g, g + 8 of the warp's 32
+        tmem_ld_16x256b_x8_async(src + (16u << 16), vb);  // rows g + 16, g + 24
+        tmem_wait_ld32(va);
+        tmem_tie32(vb);
+        if (half == 1 || piece == 1) {
+          tc_fence_before();
+          mbar_arrive(smem_u32(half == 1 ? (piece == 0 ? &bar_dq1afree : &bar_dq1bfree) : &bar_dq0free));
+        }
+        float x0[8][2], x1[8][2], x2[8][2], x3[8][2];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          x0[k][0] = __uint_as_float(va[4 * k]);
+          x0[k][1] = __uint_as_float(va[4 * k + 1]);
+          x1[k][0] = __uint_as_float(va[4 * k + 2]);
+          x1[k][1] = __uint_as_float(va[4 * k + 3]);
+          x2[k][0] = __uint_as_float(vb[4 * k]);
+          x2[k][1] = __uint_as_float(vb[4 * k + 1]);
+          x3[k][0] = __uint_as_float(vb[4 * k + 2]);
+          x3[k][1] = __uint_as_float(vb[4 * k + 3]);
+        }
+        // after the transposes lane 4 g + c writes columns 8g + 2c, +1 of each row
+        float* base = tile + static_cast<size_t>(wrow) * C::HD + half * 128 + piece * 64 + 8 * g + 2 * c;
+        drain_rowset<0>(base, x0, g, live);
+        drain_rowset<8>(base, x1, g, live);
+        drain_rowset<16>(base, x2, g, live);
+        drain_rowset<24>(base, x3, g, live);
       }
     }
   }
-
-  // warps 14, 15: idle
 
   tc_fence_before();
   __syncthreads();

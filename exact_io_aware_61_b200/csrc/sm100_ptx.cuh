@@ -150,6 +150,13 @@ FA_DEV void red_add_v4_f32(float* p, float a, float b, float c, float d) {
                : "memory");
 }
 
+// 8-byte f32 reduction at p + OFF bytes (an immediate offset, so that a run of
+// them shares one address register)
+template <int OFF>
+FA_DEV void red_add_v2_f32(float* p, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0+%3], {%1, %2};" ::"l"(p), "f"(a), "f"(b), "n"(OFF) : "memory");
+}
+
 // Move this warp's register allocation from the launch count LAUNCH to N
 // (setmaxnreg: .inc to raise it, .dec to lower it). The caller's warpgroups
 // must add up to the launch allocation, or an .inc waits forever.
@@ -391,6 +398,25 @@ FA_DEV void tmem_tie16(uint32_t (&r)[16]) {
                  "+r"(r[15])
                :
                : "memory");
+}
+
+// TMEM -> registers, 16 lanes x 64 columns in the 16x256b shape, not waited
+// (tcgen05.wait::ld before use; tmem_wait_ld32 / tmem_tie32 tie the
+// registers to it). Thread t of the warp gets, for each 8-column chunk k,
+// registers 4k, 4k+1 = lane (base + t/4), columns 8k + 2 (t % 4) and the next
+// one; registers 4k+2, 4k+3 = lane (base + 8 + t/4), the same columns: four
+// consecutive threads hold 32 contiguous bytes of a row.
+FA_DEV void tmem_ld_16x256b_x8_async(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
 }
 
 FA_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
