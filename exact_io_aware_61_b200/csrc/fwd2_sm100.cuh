@@ -51,6 +51,10 @@ struct Fwd2Cfg {
   static constexpr uint32_t TMEM_P = 384;
   static constexpr float RESCALE_THRESHOLD = 8.0f;
   static constexpr int HEAD_GROUP = 8;  // heads scheduled together (K/V stay in L2)
+  // Roles of the third warpgroup. Warp w runs on SM sub-partition w % 4,
+  // which it shares with softmax warps w % 4 and w % 4 + 4.
+  static constexpr int PRODUCER_WARP = 8;
+  static constexpr int MMA_WARP = 9;
 };
 
 struct Fwd2Params {
@@ -238,7 +242,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(smem_u32(&bar_drain), 1);
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(&tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -250,9 +254,9 @@ __global__ void __launch_bounds__(384, 1)
   if (warp >= 8) {
     set_max_regs<C::OTHER_REGS, C::LAUNCH_REGS>();
   }
-  if (warp >= 10) {
+  if (warp >= 8 && warp != C::PRODUCER_WARP && warp != C::MMA_WARP) {
     // idle warps of the third warpgroup
-  } else if (warp == 8) {
+  } else if (warp == C::PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -294,7 +298,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = max(0, v_issued - VST); j < v_issued; ++j)
         (void)mbar_wait_drain(smem_u32(&bar_vfull[j % VST]), (j / VST) & 1, p.timeout_ns);
     }
-  } else if (warp == 9) {
+  } else if (warp == C::MMA_WARP) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
@@ -515,7 +519,7 @@ __global__ void __launch_bounds__(384, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
