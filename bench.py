@@ -50,8 +50,8 @@ SPEC_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor peak, vendor figure (context
 PROFILED = {
     # ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum,
     #     sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active at the benchmark shape
-    "bwd_main": {"src": "c7a133affb2181e8", "dram_bytes": 826_841_088 + 499_585_024, "tensor_pipe_active_pct": 41.80},
-    "fwd": {"src": "c7a133affb2181e8", "dram_bytes": 403_137_536 + 115_962_880, "tensor_pipe_active_pct": 50.90},
+    "bwd_main": {"src": "a8dc487b9b750668", "dram_bytes": 825_466_112 + 498_840_832, "tensor_pipe_active_pct": 41.76},
+    "fwd": {"src": "a8dc487b9b750668", "dram_bytes": 403_888_384 + 116_158_464, "tensor_pipe_active_pct": 51.00},
 }
 
 
