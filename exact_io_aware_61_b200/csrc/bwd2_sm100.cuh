@@ -30,9 +30,10 @@
 //   warp 13     TMEM allocator and MMA issuer; warps 14, 15 idle
 // MMA order per step t (query tile):
 //   dP^T(t) [once dQ(t-1) left TMEM], dV += P^T dO, S^T(t+1) [over P^T(t),
-//   which dV(t) has read], dK += dS^T Q, dQ(t) [into the dP^T columns]: the
+//   which dV(t) has read], dQ(t) [into the dP^T columns], dK += dS^T Q: the
 //   next step's scores are ready while the compute warpgroups form dS^T(t),
-//   and the drain empties dQ(t) while they work on step t+1.
+//   dQ(t) reaches the drain without waiting for dK(t), and the drain empties
+//   dQ(t) while they work on step t+1.
 // TMEM: S^T / P^T at 0, dP^T / dQ at 128, dV at 256, dK at 256 + d.
 // Every MMA runs 128 x 128 (or 128 x d) per instruction, the size at which
 // operands in shared memory and in tensor memory both keep the tensor core
@@ -349,20 +350,23 @@ __global__ void __launch_bounds__(512, 1)
           tc_fence_after();
           issue_s(t + 1);
         }
-        // dK += dS^T Q (A = dS^T in shared memory, keys x queries, K-major);
-        // dQ = dS K (the same buffer read as dS, queries x keys, M-major)
+        // dQ = dS K (A = dS^T's shared-memory tile read as queries x keys,
+        // M-major), then dK += dS^T Q (the same tile as keys x queries,
+        // K-major). dQ goes first: the drain, and through it dP^T(t+1), wait
+        // for it, while nothing waits for dK before the next step's dK.
         if (!mbar_wait(smem_u32(&bar_dsfull), t & 1, wc)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + C::T_DK, sdesc_sw128(sDS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                      sdesc_sw128(qst + kk * 2048, 16384, 1024), id_kmn, (t > 0 || kk > 0));
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ss(tmem + C::T_DP, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
                       sdesc_sw128(sK + kk * 2048, 16384, 1024), id_mnmn, kk > 0);
-        mma_commit(smem_u32(&bar_qempty[sq]));
         mma_commit(smem_u32(&bar_dqfull));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(tmem + C::T_DK, sdesc_sw128(sDS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                      sdesc_sw128(qst + kk * 2048, 16384, 1024), id_kmn, (t > 0 || kk > 0));
+        // the Q stage and the dS tile are free once dK(t) has completed
+        mma_commit(smem_u32(&bar_qempty[sq]));
       }
       // bar_final completes once every MMA issued above has completed (on
       // the normal path and after a bounded wait gave up alike); no MMA may
@@ -442,7 +446,9 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_before();
       mbar_arrive(smem_u32(&bar_pfull));
       // ---- dS^T = P^T (dP^T - D) * scale -> shared memory
-      if (t > 0 && !warp_wait(smem_u32(&bar_dqfull), (t - 1) & 1, wc)) { ok = false; break; }  // dS(t-1) consumed
+      // dS(t-1) consumed: dK(t-1), the last MMA to read it, completes the
+      // release of Q stage (t-1) % QST
+      if (t > 0 && !warp_wait(smem_u32(&bar_qempty[(t - 1) % QST]), ((t - 1) / QST) & 1, wc)) { ok = false; break; }
       if (!warp_wait(smem_u32(&bar_dpfull), t & 1, wc)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
