@@ -50,8 +50,8 @@ SPEC_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor peak, vendor figure (context
 PROFILED = {
     # ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum,
     #     sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active at the benchmark shape
-    "bwd_main": {"src": "a8dc487b9b750668", "dram_bytes": 825_466_112 + 498_840_832, "tensor_pipe_active_pct": 41.76},
-    "fwd": {"src": "a8dc487b9b750668", "dram_bytes": 403_888_384 + 116_158_464, "tensor_pipe_active_pct": 51.00},
+    "bwd_main": {"src": "c441493b0815a76b", "dram_bytes": 821_930_240 + 501_082_624, "tensor_pipe_active_pct": 41.97},
+    "fwd": {"src": "c441493b0815a76b", "dram_bytes": 402_914_048 + 115_728_384, "tensor_pipe_active_pct": 50.99},
 }
 
 
