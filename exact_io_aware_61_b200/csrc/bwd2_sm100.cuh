@@ -54,8 +54,11 @@ struct Bwd2Cfg {
   static constexpr int DOST = HD == 64 ? 2 : 1;
   static constexpr int QSTAGE_BYTES = TILE + 1024;
   static constexpr int DS_BYTES = 128 * 128 * 2;
-  // one 128-row x 32-column f32 box of the dQ tile, staged for a TMA reduce-add
-  static constexpr int DQ_STAGE_BYTES = 128 * 32 * 4;
+  // dQ staging: one 32-row x 32-column f32 box per drain warp (its own rows
+  // of the tile), each added to the accumulator with a TMA reduce-add
+  static constexpr int DQ_BOX_ROWS = 32;
+  static constexpr int DQ_BOX_BYTES = DQ_BOX_ROWS * 32 * 4;
+  static constexpr int DQ_STAGE_BYTES = 4 * DQ_BOX_BYTES;
   static constexpr int SMEM_BYTES =
       1024 + 2 * TILE + QST * QSTAGE_BYTES + DOST * TILE + DS_BYTES + DQ_STAGE_BYTES;
   static constexpr int THREADS = 512;
@@ -515,20 +518,18 @@ __global__ void __launch_bounds__(512, 1)
   } else {
     set_max_regs<C::DRAIN_REGS, C::LAUNCH_REGS>();
     // ------------------------------------------------------- dQ warpgroup
-    // Thread tid holds query row q0 + tid of the dQ tile (TMEM lane = row).
+    // Thread i of the warpgroup holds query row q0 + i of the dQ tile (TMEM lane = row).
     // The whole tile is loaded into registers and its columns released to
-    // dP^T(t+1) at once; then, 32 head-dim columns at a time, the rows are
-    // written to a 128-byte-swizzled staging box (one 16-byte vector per
-    // store) and added to the f32 accumulator with a TMA tensor reduce-add,
-    // which also drops rows past N.
-    //
-    // The four warps synchronise with a hardware named barrier. Every warp
-    // runs the same number of barriers whatever happens (a bounded wait that
-    // gives up only clears `ok`, which skips work, never barriers), so a
-    // timeout cannot leave a warp waiting at a barrier for ever.
-    const int tid = threadIdx.x - 256;
-    const uint32_t lane_base = ((warp & 3) * 32u) << 16;
-    uint8_t* stage_row = gbase + (sDQ - base) + tid * 128;
+    // dP^T(t+1) at once; then, 32 head-dim columns at a time, each warp
+    // writes its 32 rows to its own 128-byte-swizzled staging box (one
+    // 16-byte vector per store) and adds the box to the f32 accumulator with
+    // a TMA tensor reduce-add, which also drops rows past N. The four warps
+    // run independently: while the TMA unit reads one warp's box at the rate
+    // the L2 takes the reductions, the other warps fill theirs.
+    const int dw = warp & 3;  // rows 32 dw .. 32 dw + 31 of the tile
+    const uint32_t lane_base = (dw * 32u) << 16;
+    const uint32_t box = sDQ + dw * C::DQ_BOX_BYTES;
+    uint8_t* stage_row = gbase + (box - base) + lane * 128;
     bool ok = true;
     for (int t = 0; t < steps; ++t) {
       int bhq, q0;
@@ -547,25 +548,25 @@ __global__ void __launch_bounds__(512, 1)
       }
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
-        if (tid == 0) bulk_wait_group_read<0>();  // the last reduce has read the staging box
-        named_bar_sync(1, 128);
+        if (lane == 0) bulk_wait_group_read<0>();  // this warp's last reduce has read its box
+        __syncwarp();
         if (ok) {
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(stage_row + ((u ^ (tid & 7)) * 16)) =
+            *reinterpret_cast<uint4*>(stage_row + ((u ^ (lane & 7)) * 16)) =
                 make_uint4(rr[c][4 * u], rr[c][4 * u + 1], rr[c][4 * u + 2], rr[c][4 * u + 3]);
         }
         fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (tid == 0 && ok) {
+        __syncwarp();
+        if (lane == 0 && ok) {
           int qy, qz;
-          q_yz(bhq, q0, qy, qz);
-          tma_reduce_add_3d(&tm_dq, sDQ, c * 32, qy, qz);
+          q_yz(bhq, q0 + 32 * dw, qy, qz);
+          tma_reduce_add_3d(&tm_dq, box, c * 32, qy, qz);
           bulk_commit_group();
         }
       }
     }
-    if (tid == 0) bulk_wait_all();
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();

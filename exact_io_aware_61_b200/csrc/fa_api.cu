@@ -518,7 +518,8 @@ int plan_bwd(BwdPlan* pl, unsigned stages, const void* q, const void* k, const v
     if (rc == FA_OK) rc = make_map(&pl->mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_kv, 64, 128);
     if (rc == FA_OK) rc = make_map(&pl->mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, N, rows_q, 64, 128);
     if (rc == FA_OK)
-      rc = make_map(&pl->mdq, pl->w.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, N, rows_q, 32, 128);
+      rc = make_map(&pl->mdq, pl->w.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, N, rows_q, 32,
+                    fa::Bwd2Cfg<HD>::DQ_BOX_ROWS);
     if (rc != FA_OK) return rc;
     fa::Bwd2Params& mp = pl->mp;
     mp.ws_delta = pl->w.delta;
@@ -640,7 +641,8 @@ int run_bwd_varlen(const void* q, const void* k, const void* v, const void* o, c
   if (rc == FA_OK) rc = make_map3(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hkv, total_k, 64, 1, 128);
   if (rc == FA_OK) rc = make_map3(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hkv, total_k, 64, 1, 128);
   if (rc == FA_OK) rc = make_map3(&mdo, dO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HD, Hq, total_q, 64, 1, 128);
-  if (rc == FA_OK) rc = make_map3(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, Hq, total_q, 32, 1, 128);
+  if (rc == FA_OK)
+    rc = make_map3(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HD, Hq, total_q, 32, 1, fa::Bwd2Cfg<HD>::DQ_BOX_ROWS);
   if (rc != FA_OK) return rc;
   fa::BwdPrepVarlenParams pp;
   pp.o = static_cast<const __nv_bfloat16*>(o);
