@@ -50,8 +50,8 @@ SPEC_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor peak, vendor figure (context
 PROFILED = {
     # ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum,
     #     sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active at the benchmark shape
-    "bwd_main": {"src": "aef54d5051bedb21", "dram_bytes": 826_123_520 + 499_622_144, "tensor_pipe_active_pct": 48.59},
-    "fwd": {"src": "aef54d5051bedb21", "dram_bytes": 403_515_392 + 116_814_848, "tensor_pipe_active_pct": 50.99},
+    "bwd_main": {"src": "37c76f4c2b2b572a", "dram_bytes": 825_743_872 + 498_451_456, "tensor_pipe_active_pct": 48.71},
+    "fwd": {"src": "37c76f4c2b2b572a", "dram_bytes": 404_009_984 + 116_269_056, "tensor_pipe_active_pct": 51.60},
 }
 
 

@@ -324,6 +324,18 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; ok && j < n_max; ++j) {
         const int s = j % VST;
         bool v_ready = false, k_next_ready = false;
+        if constexpr (!C::SEP_P) {
+          // V(j) and K(j+1) were loaded at least a key tile ago (their stages
+          // were released by earlier iterations): wait for them here, while the
+          // softmax still works on S(j), not between a tile's P and its MMAs
+          if (!mbar_wait(smem_u32(&bar_vfull[s]), (j / VST) & 1, wc)) break;
+          v_ready = true;
+          if (j + 1 < n_max) {
+            if (!mbar_wait(smem_u32(&bar_kfull[(j + 1) % KST]), ((j + 1) / KST) & 1, wc)) break;
+            k_next_ready = true;
+          }
+          tc_fence_after();
+        }
         if constexpr (C::SEP_P) {
           // S(j+1) of each tile as soon as its softmax has read S(j); P(j)
           // has its own columns, so it does not wait for P(j)V(j)
