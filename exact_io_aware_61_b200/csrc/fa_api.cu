@@ -72,6 +72,19 @@ int check_device(int* dev_out) {
   return FA_OK;
 }
 
+// Every configuration's dynamic shared memory fits the 227 KB (232,448 bytes)
+// a block can opt into, with 1 KB left for its static barriers.
+constexpr int kMaxDynamicSmem = 232448 - 1024;
+static_assert(fa::Fwd2Cfg<64>::SMEM_BYTES <= kMaxDynamicSmem && fa::Fwd2Cfg<128>::SMEM_BYTES <= kMaxDynamicSmem,
+              "two-tile forward shared memory");
+static_assert(fa::FwdCfg<256>::SMEM_BYTES <= kMaxDynamicSmem && fa::FwdCfg<64, true>::SMEM_BYTES <= kMaxDynamicSmem &&
+                  fa::FwdCfg<128, true>::SMEM_BYTES <= kMaxDynamicSmem &&
+                  fa::FwdCfg<256, true>::SMEM_BYTES <= kMaxDynamicSmem,
+              "one-tile forward shared memory");
+static_assert(fa::Bwd2Cfg<64>::SMEM_BYTES <= kMaxDynamicSmem && fa::Bwd2Cfg<128>::SMEM_BYTES <= kMaxDynamicSmem,
+              "backward shared memory");
+static_assert(fa::Bwd256Cfg::SMEM_BYTES <= kMaxDynamicSmem, "d = 256 backward shared memory");
+
 // Opt every kernel into its dynamic shared memory, once per device.
 int prepare_kernels(int dev) {
   static std::mutex mu;
